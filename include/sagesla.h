@@ -1,0 +1,146 @@
+/*
+ * sagesla.h - SageSLA attention forward for NVIDIA B200 (sm_100a), C ABI.
+ *
+ * SageSLA stacks two attention accelerations described in "TurboDiffusion Demystified:
+ * How It Achieves 100x Faster Video Generation":
+ *   - section "Pillar One: Low-Bit Attention Acceleration - SageAttention": Q K^T in
+ *     INT8 on tensor cores, with K smoothed against outliers;
+ *   - section "Pillar Two: Sparse-Linear Attention - SLA": per query block only the
+ *     most important key blocks get exact attention (--sla_topk 0.1 keeps 10%, section
+ *     "Hands-On Tutorial"), a light linear-attention term covers the middle, the rest is
+ *     skipped.
+ *
+ * Per (batch, head), with 64-token blocks and head dim d = 128:
+ *   (1) mu = per-channel mean of K over the N real tokens; K~ = K - mu.
+ *   (2) Q~ = Q * sm_scale (sm_scale = fl32(1/sqrt(d)), passed in).
+ *   (3) Q~ and K~ quantized per block to symmetric INT8: s = max|x|/127,
+ *       x8 = clamp(rint(x/s), -127, 127), round half to even.
+ *   (4) logit l_ij = mean(Q~_i) . mean(K~_j) in fp32; per query-block row the top
+ *       k_c = ceil(rho*nB) key blocks are critical, the bottom n_neg = floor(nu*nB)
+ *       negligible, the rest (m) marginal; equal logits rank the lower index first.
+ *   (5) critical blocks: online-softmax attention, scores (q8.k8) * s_q * s_k,
+ *       P rounded to bf16 for P.V with fp32 accumulation.
+ *   (6) marginal blocks: phi(x) = elu(x)+1, h_j = phi(K~_j)^T V_j, z_j = phi(K~_j)^T 1,
+ *       H_i = sum_marg h_j, Z_i = sum_marg z_j, O_l = phi(Q~) H_i / (phi(Q~) . Z_i).
+ *   (7) O = O_s + O_l, rounded to bf16.
+ *
+ * Conventions for every call below.
+ *   - All tensor pointers are DEVICE pointers, contiguous, row-major, 16-byte aligned.
+ *     The caller owns every buffer; the library allocates, frees and synchronizes
+ *     nothing (except sagesla_check_status, which synchronizes the stream).
+ *   - nB = ceil(N/64), Npad = 64*nB, nBp = 64*ceil(nB/64) (pitch of the mask rows).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - Return value: SAGESLA_OK, or an error code from host-side validation (nothing is
+ *     launched), or SAGESLA_ERR_CUDA if a launch failed. Device-side timeouts of bounded
+ *     waits are recorded in the workspace status word; read it with
+ *     sagesla_check_status.
+ *   - Outputs must not alias inputs. Only d = 128 is supported (else UNSUPPORTED).
+ *   - Calls are re-entrant across streams if each stream uses its own workspace.
+ */
+#ifndef SAGESLA_H
+#define SAGESLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SAGESLA_OK = 0,
+  SAGESLA_ERR_INVALID_ARG = 1, /* null pointer, misalignment, bad ratio or size      */
+  SAGESLA_ERR_UNSUPPORTED = 2, /* valid but not implemented (d != 128, sizes > max)  */
+  SAGESLA_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed               */
+  SAGESLA_ERR_TIMEOUT = 4      /* a bounded device wait gave up (see check_status)   */
+} sagesla_status;
+
+typedef struct {
+  int B; /* batch                       */
+  int H; /* heads                       */
+  int N; /* tokens per (batch, head)    */
+  int d; /* head dim; must be 128       */
+} sagesla_shape;
+
+/* Block counts for one query-block row (step 4).
+ * k_c = ceil(rho*nB) (>= 1), n_neg = floor(nu*nB) capped at nB-k_c, m = nB-k_c-n_neg;
+ * a product within 1e-9 (relative) of an integer counts as that integer.
+ * Requires 0 < rho <= 1 and 0 <= nu < 1. Any output pointer may be NULL. */
+int sagesla_counts(const sagesla_shape* shape, double rho, double nu,
+                   int* nB, int* k_c, int* n_neg, int* m);
+
+/* Bytes of device workspace that prepare and forward need for this shape (the same
+ * buffer serves both). It holds the status word, the per-block channel partial sums
+ * of step (1), H_i (bf16 [B,H,nB,d,d]), Z_i (fp32 [B,H,nB,d]) and the linear-branch
+ * output (bf16 [B,H,N,d]). Returns 0 for an invalid shape. */
+size_t sagesla_workspace_bytes(const sagesla_shape* shape);
+
+/* Zero the workspace status word (enqueued on stream). Call once after allocating. */
+int sagesla_reset_status(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Steps (1)-(3), the block means of (4) and the linear states of (6).
+ * Inputs : q, k, v  bf16 [B,H,N,d]; sm_scale = fl32(1/sqrt(d)) computed by the caller.
+ * Outputs: q8, k8      int8 [B,H,Npad,d] (padded rows written as 0)
+ *          q_scale, k_scale fp32 [B,H,nB]
+ *          k_mean       fp32 [B,H,d]   (mu)
+ *          q_bar, k_bar fp32 [B,H,nB,d] (block means of Q~ and K~ over real tokens)
+ *          h            bf16 [B,H,nB,d,d]  h_j[c][e] = sum_t phi(K~_t[c]) V_t[e]
+ *          z            fp32 [B,H,nB,d]    z_j[c]    = sum_t phi(K~_t[c])
+ * INT8 codes, scales, mu and the block means are bit-exact with a fixed summation
+ * order (sequential in token order within a block, then over blocks). */
+int sagesla_prepare(const sagesla_shape* shape, const void* q, const void* k,
+                    const void* v, float sm_scale, int8_t* q8, int8_t* k8,
+                    float* q_scale, float* k_scale, float* k_mean, float* q_bar,
+                    float* k_bar, void* h, float* z, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* Step (4): block logits, ranking and the per-row block lists.
+ * Inputs : q_bar, k_bar fp32 [B,H,nB,d]; rho, nu as in sagesla_counts.
+ * Outputs: crit_idx int32 [B,H,nB,k_c]  ascending critical key blocks per row
+ *          marg_idx int32 [B,H,nB,m]    ascending marginal key blocks per row (may be
+ *                                       NULL when m == 0)
+ *          marg_mask bf16 [B,H,nB,nBp]  1.0 where block j is marginal for row i, 0
+ *                                       elsewhere (including the pitch padding)
+ *          logits   fp32 [B,H,nB,nB]    optional (NULL = not written)
+ * Logits use a fixed fp32 order (acc = 0; acc = fl32(acc + fl32(qbar*kbar)) for
+ * c = 0..d-1), so the lists are bit-exact against any implementation that follows it. */
+int sagesla_select(const sagesla_shape* shape, const float* q_bar, const float* k_bar,
+                   double rho, double nu, int32_t* crit_idx, int32_t* marg_idx,
+                   void* marg_mask, float* logits, void* stream);
+
+/* Steps (5)-(7).
+ * Inputs : q bf16 [B,H,N,d] (phi(Q~) is recomputed from it), sm_scale, and the
+ *          outputs of prepare and select; k_c and m must be the counts of select.
+ *          v bf16 [B,H,N,d].
+ * Output : out bf16 [B,H,N,d] (rows t >= N are not touched).
+ * workspace: at least sagesla_workspace_bytes(shape) bytes. */
+int sagesla_forward(const sagesla_shape* shape, const void* q, float sm_scale,
+                    const int8_t* q8, const int8_t* k8, const float* q_scale,
+                    const float* k_scale, const void* v, const int32_t* crit_idx, int k_c,
+                    const void* marg_mask, const int32_t* marg_idx, int m, const void* h,
+                    const float* z, void* out, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/* Synchronize `stream`, then return the workspace status word: SAGESLA_OK, or
+ * SAGESLA_ERR_TIMEOUT if a bounded device wait gave up (the affected output is
+ * invalid), or SAGESLA_ERR_CUDA if the stream reported an error. */
+int sagesla_check_status(const void* workspace, void* stream);
+
+/* Launch tracing (diagnostics). While enabled, every kernel launch made by this library
+ * is bracketed by a pair of CUDA events recorded on its launch stream. Process-global
+ * state, guarded by a mutex; meant for benchmarking, not for concurrent production use. */
+int sagesla_trace_enable(int on);
+
+/* Synchronize on the recorded events and write one line per kernel name,
+ * "<kernel> <launches> <total_ms>\n", into buf (NUL-terminated, truncated to len); the
+ * records are then cleared. Returns SAGESLA_OK, SAGESLA_ERR_CUDA if an event failed, or
+ * SAGESLA_ERR_INVALID_ARG if buf was too small. */
+int sagesla_trace_read(char* buf, size_t len);
+
+/* Human-readable name of a status code (static string). */
+const char* sagesla_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SAGESLA_H */

@@ -1,0 +1,299 @@
+// linear.cu - the linear-attention branch for marginal key blocks.
+//
+// Method: "TurboDiffusion Demystified", section "Pillar Two: Sparse-Linear Attention -
+// SLA": the key blocks that are neither kept exactly nor skipped are covered by a light
+// linear-attention term. With phi(x) = elu(x) + 1 and the per-key-block states
+// h_j = phi(K~_j)^T V_j, z_j = phi(K~_j)^T 1 written by prepare:
+//   H_i = sum_{j marginal for i} h_j,  Z_i = sum_{j marginal} z_j,
+//   O_l[t] = phi(Q~_t)^T H_i / (phi(Q~_t) . Z_i).
+//
+// Kernels:
+//   hgemm_kernel   H = M . h per head, M the 0/1 marginal mask [nB x nBp] and h viewed as
+//                  [nB x d*d]: a tcgen05 bf16 GEMM (fp32 accumulation in TMEM), 128x128
+//                  output tiles, TMA-fed 3-stage pipeline, bf16 output.
+//   zsum_kernel    Z_i = sum of z_j over the marginal list, fp32, ascending j.
+//   linout_kernel  per pair of query blocks: phi(Q~) (recomputed from Q, bf16) times H_i
+//                  on tcgen05 (M = 128 rows = both blocks, one MMA chain per block),
+//                  divided by phi(Q~) . Z_i; bf16 O_l for the attention epilogue.
+#include "sagesla_internal.h"
+#include "sm100_primitives.cuh"
+
+namespace sgs {
+namespace {
+
+// ------------------------------------------------------------------ H = M . h
+constexpr int kGemmStages = 3;
+constexpr int kGemmStageBytes = 16384 + 16384;
+constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + 1024 + 256;
+
+__global__ void __launch_bounds__(128) hgemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                                                    const __grid_constant__ CUtensorMap tmB,
+                                                    __nv_bfloat16* __restrict__ Hout, int nB,
+                                                    int* status) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemmStages * kGemmStageBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kGemmStages;
+  uint64_t* done = bars + 2 * kGemmStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  __shared__ int abort_flag;
+
+  const int nt = blockIdx.x, mt = blockIdx.y, bh = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nK = (nB + 63) / 64;
+
+  if (tid == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < kGemmStages; ++s) {
+      mbar_init(smem_u32(full + s), 1);
+      mbar_init(smem_u32(empty + s), 1);
+    }
+    mbar_init(smem_u32(done), 1);
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 128);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t taddr = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    for (int kb = 0; kb < nK; ++kb) {
+      const int s = kb % kGemmStages;
+      if (kb >= kGemmStages &&
+          !mbar_wait(smem_u32(empty + s), ((kb / kGemmStages) - 1) & 1, &abort_flag, status))
+        break;
+      const uint32_t sa = smem_u32(smem + s * kGemmStageBytes);
+      const uint32_t sb = sa + 16384;
+      mbar_expect_tx(smem_u32(full + s), kGemmStageBytes);
+      tma_load_3d(sa, &tmA, smem_u32(full + s), kb * 64, mt * 128, bh);
+      tma_load_3d(sb, &tmB, smem_u32(full + s), nt * 128, kb * 64, bh);
+      tma_load_3d(sb + 8192, &tmB, smem_u32(full + s), nt * 128 + 64, kb * 64, bh);
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = make_idesc(1, 1, 0, 1, 128, 128);
+    bool ok = true;
+    for (int kb = 0; kb < nK && ok; ++kb) {
+      const int s = kb % kGemmStages;
+      ok = mbar_wait(smem_u32(full + s), (kb / kGemmStages) & 1, &abort_flag, status);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t sa = smem_u32(smem + s * kGemmStageBytes);
+      const uint32_t sb = sa + 16384;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(taddr, make_sdesc(sa + kk * 32, 16, 1024), make_sdesc(sb + kk * 2048, 8192, 1024),
+                 idesc, (kb | kk) != 0);
+      mma_commit(smem_u32(empty + s));
+    }
+    mma_commit(smem_u32(done));
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(smem_u32(done), 0, &abort_flag, status);
+  tc_fence_after();
+  if (ok) {
+    const int i = mt * 128 + 32 * warp + lane;
+    __nv_bfloat16* dst = Hout + (static_cast<size_t>(bh) * nB + i) * (kHeadDim * kHeadDim) + nt * 128;
+#pragma unroll
+    for (int cchunk = 0; cchunk < 4; ++cchunk) {
+      uint32_t r[32];
+      tmem_ld32_sync(taddr + (static_cast<uint32_t>(32 * warp) << 16) + 32 * cchunk, r);
+      if (i < nB) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cchunk);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          d4[q] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
+                             pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
+                             pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
+                             pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(taddr, 128);
+}
+
+// ------------------------------------------------------------------ Z_i
+__global__ void __launch_bounds__(128) zsum_kernel(const float* __restrict__ z,
+                                                   const int32_t* __restrict__ marg,
+                                                   float* __restrict__ Z, int nB, int m) {
+  const int i = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
+  const int32_t* ml = marg + (static_cast<size_t>(bh) * nB + i) * m;
+  const float* zb = z + static_cast<size_t>(bh) * nB * kHeadDim + c;
+  float acc = 0.f;
+  for (int t = 0; t < m; ++t) acc += zb[static_cast<size_t>(ml[t]) * kHeadDim];
+  Z[(static_cast<size_t>(bh) * nB + i) * kHeadDim + c] = acc;
+}
+
+// ------------------------------------------------------------------ O_l
+constexpr int kLinSmem = 32768 + 65536 + 1024 + 256;
+
+__global__ void __launch_bounds__(128) linout_kernel(const __grid_constant__ CUtensorMap tmH,
+                                                     const __nv_bfloat16* __restrict__ q,
+                                                     const float* __restrict__ Z, float c_s,
+                                                     __nv_bfloat16* __restrict__ Ol, int N,
+                                                     int nB, int* status) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* sA = smem;            // phi(Q~): 2 column blocks x 128 rows x 128 B
+  unsigned char* sH = smem + 32768;    // H_i0, H_i1: each 2 e-groups x 128 c rows x 128 B
+  uint64_t* hfull = reinterpret_cast<uint64_t*>(smem + 32768 + 65536);
+  uint64_t* mdone = hfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + 1);
+  __shared__ int abort_flag;
+
+  const int pr = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int i0 = 2 * pr;
+  const bool two = (i0 + 1) < nB;
+  if (tid == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(hfull), 1);
+    mbar_init(smem_u32(mdone), 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t taddr = *tmem_slot;
+
+  if (tid == 0) {
+    mbar_expect_tx(smem_u32(hfull), two ? 65536 : 32768);
+    for (int b = 0; b < (two ? 2 : 1); ++b) {
+      const uint32_t dst = smem_u32(sH) + b * 32768;
+      tma_load_3d(dst, &tmH, smem_u32(hfull), 0, (i0 + b) * 128, bh);
+      tma_load_3d(dst + 16384, &tmH, smem_u32(hfull), 64, (i0 + b) * 128, bh);
+    }
+  }
+
+  // phi(Q~) row r and its denominator phi(Q~).Z_i (with the bf16-rounded phi values the
+  // tensor core sees).
+  const int r = tid;
+  const int i = i0 + (r >> 6);
+  const int t = i * 64 + (r & 63);
+  const bool valid = (i < nB) && (t < N);
+  float den = 1.f;
+  {
+    const __nv_bfloat16* qr = q + (static_cast<size_t>(bh) * N + (valid ? t : 0)) * kHeadDim;
+    const float* zr = Z + (static_cast<size_t>(bh) * nB + (i < nB ? i : 0)) * kHeadDim;
+    float dacc = 0.f;
+#pragma unroll
+    for (int cb = 0; cb < 16; ++cb) {  // 8 channels per chunk
+      uint32_t w[4] = {0, 0, 0, 0};
+      if (valid) {
+        const uint4 u = *reinterpret_cast<const uint4*>(qr + 8 * cb);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(b2[e]);
+          const float x0 = __fmul_rn(f.x, c_s), x1 = __fmul_rn(f.y, c_s);
+          const float p0 = x0 > 0.f ? x0 + 1.f : expf(x0);
+          const float p1 = x1 > 0.f ? x1 + 1.f : expf(x1);
+          w[e] = pack_bf16x2(p0, p1);
+          const float2 pr2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
+          dacc = fmaf(pr2.x, zr[8 * cb + 2 * e], dacc);
+          dacc = fmaf(pr2.y, zr[8 * cb + 2 * e + 1], dacc);
+        }
+      }
+      st_shared_v4(smem_u32(sA) + (cb >> 3) * 16384 + sw128_offset(r, cb & 7), w[0], w[1], w[2], w[3]);
+    }
+    if (valid) den = dacc;
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  if (tid == 0) {
+    bool ok = mbar_wait(smem_u32(hfull), 0, &abort_flag, status);
+    tc_fence_after();
+    if (ok) {
+      constexpr uint32_t idesc = make_idesc(1, 1, 0, 1, 128, 128);
+      for (int b = 0; b < (two ? 2 : 1); ++b) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = make_sdesc(smem_u32(sA) + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = make_sdesc(smem_u32(sH) + b * 32768 + kk * 2048, 16384, 1024);
+          mma_bf16(taddr + 128 * b, a, bd, idesc, kk > 0);
+        }
+      }
+    }
+    mma_commit(smem_u32(mdone));
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(smem_u32(mdone), 0, &abort_flag, status);
+  tc_fence_after();
+  if (ok && (i < nB)) {  // warp-uniform: rows 0-63 -> warps 0,1; rows 64-127 -> warps 2,3
+    const int half = warp >> 1;
+    const float inv = 1.f / den;
+    __nv_bfloat16* dst = Ol + (static_cast<size_t>(bh) * N + (valid ? t : 0)) * kHeadDim;
+#pragma unroll
+    for (int cchunk = 0; cchunk < 4; ++cchunk) {
+      uint32_t rr[32];
+      tmem_ld32_sync(taddr + (static_cast<uint32_t>(32 * warp) << 16) + 128 * half + 32 * cchunk, rr);
+      if (valid) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cchunk);
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq)
+          d4[qq] = make_uint4(
+              pack_bf16x2(__uint_as_float(rr[8 * qq]) * inv, __uint_as_float(rr[8 * qq + 1]) * inv),
+              pack_bf16x2(__uint_as_float(rr[8 * qq + 2]) * inv, __uint_as_float(rr[8 * qq + 3]) * inv),
+              pack_bf16x2(__uint_as_float(rr[8 * qq + 4]) * inv, __uint_as_float(rr[8 * qq + 5]) * inv),
+              pack_bf16x2(__uint_as_float(rr[8 * qq + 6]) * inv, __uint_as_float(rr[8 * qq + 7]) * inv));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(taddr, 256);
+}
+
+}  // namespace
+
+cudaError_t launch_linear(const Dims& g, const void* q, float sm_scale, const void* mask,
+                          const int32_t* marg, int m, const void* h, const float* z, char* ws,
+                          cudaStream_t st) {
+  if (m == 0) return cudaSuccess;
+  const WsLayout L = ws_layout(g);
+  int* status = reinterpret_cast<int*>(ws + L.status);
+  __nv_bfloat16* Hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.Hbuf);
+  float* Zbuf = reinterpret_cast<float*>(ws + L.Zbuf);
+  __nv_bfloat16* Ol = reinterpret_cast<__nv_bfloat16*>(ws + L.Ol);
+
+  CUtensorMap tmA, tmB, tmH;
+  if (!make_tmap_3d(&tmA, mask, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.nBp, g.nB, g.BH, 64, 128) ||
+      !make_tmap_3d(&tmB, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim * kHeadDim, g.nB, g.BH, 64,
+                    64) ||
+      !make_tmap_3d(&tmH, Hbuf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim,
+                    static_cast<uint64_t>(g.nB) * kHeadDim, g.BH, 64, 128))
+    return cudaErrorInvalidValue;
+
+  cudaError_t e = cudaFuncSetAttribute(hgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(linout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem);
+  if (e != cudaSuccess) return e;
+
+  {
+    TraceScope ts_("hgemm_kernel", st);
+    hgemm_kernel<<<dim3(kHeadDim * kHeadDim / 128, (g.nB + 127) / 128, g.BH), 128, kGemmSmem, st>>>(
+      tmA, tmB, Hbuf, g.nB, status);
+  }
+  {
+    TraceScope ts_("zsum_kernel", st);
+    zsum_kernel<<<dim3(g.nB, g.BH), 128, 0, st>>>(z, marg, Zbuf, g.nB, m);
+  }
+  {
+    TraceScope ts_("linout_kernel", st);
+    linout_kernel<<<dim3((g.nB + 1) / 2, g.BH), 128, kLinSmem, st>>>(
+      tmH, static_cast<const __nv_bfloat16*>(q), Zbuf, sm_scale, Ol, g.N, g.nB, status);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace sgs

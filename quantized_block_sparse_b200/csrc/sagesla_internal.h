@@ -1,0 +1,66 @@
+// sagesla_internal.h - launch entry points shared between the kernel files and the C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sgs {
+
+constexpr int kBlock = 64;     // tokens per quantization / sparsity block
+constexpr int kHeadDim = 128;  // supported head dim
+constexpr int kStatusTimeoutBit = 4;  // device status word bit for a timed-out wait
+
+struct Dims {
+  int B, H, N;
+  int BH;    // B*H
+  int nB;    // ceil(N/64)
+  int Npad;  // 64*nB
+  int nBp;   // mask row pitch: 64*ceil(nB/64)
+};
+
+// Workspace carve-up (byte offsets, 256-aligned).
+struct WsLayout {
+  size_t status;     // int32[64]
+  size_t mu_part;    // fp32 [BH, nB, d]   per-block channel sums of K
+  size_t Hbuf;       // bf16 [BH, nB, d, d]
+  size_t Zbuf;       // fp32 [BH, nB, d]
+  size_t Ol;         // bf16 [BH, N, d]
+  size_t total;
+};
+WsLayout ws_layout(const Dims& g);
+
+// prepare.cu
+cudaError_t launch_prepare(const Dims& g, const void* q, const void* k, const void* v,
+                           float sm_scale, int8_t* q8, int8_t* k8, float* q_scale,
+                           float* k_scale, float* k_mean, float* q_bar, float* k_bar, void* h,
+                           float* z, char* ws, cudaStream_t st);
+// select.cu
+cudaError_t launch_select(const Dims& g, const float* q_bar, const float* k_bar, int k_c,
+                          int n_neg, int m, int32_t* crit, int32_t* marg, void* mask,
+                          float* logits, cudaStream_t st);
+// linear.cu
+cudaError_t launch_linear(const Dims& g, const void* q, float sm_scale, const void* mask,
+                          const int32_t* marg, int m, const void* h, const float* z, char* ws,
+                          cudaStream_t st);
+// attention.cu
+cudaError_t launch_attention(const Dims& g, const int8_t* q8, const int8_t* k8,
+                             const float* q_scale, const float* k_scale, const void* v,
+                             const int32_t* crit, int k_c, int m, void* out, char* ws,
+                             cudaStream_t st);
+
+// Opt-in launch tracing (api.cu): while enabled, a CUDA event pair is recorded on the
+// launch stream around every kernel launch, so per-kernel device time can be read back.
+struct TraceScope {
+  TraceScope(const char* name, cudaStream_t st);
+  ~TraceScope();
+  int slot;
+  cudaStream_t stream;
+};
+
+// tensor maps (api.cu)
+bool make_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
+                  uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0, uint32_t box1);
+
+}  // namespace sgs

@@ -1,0 +1,120 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Bit-exact: INT8 codes, scales, mu, block means, logits and block lists (near-ties are
+counted, never expected here since the logits are bit-exact). Tolerance: the output,
+cos >= 0.9995 and max error <= 2e-2 * max|O_ref| against the oracle's quantized path;
+cos >= 0.99 against fp64 unquantized attention with the same blocks.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from quantized_block_sparse_b200.inputs import WORKLOADS, make_qkv, make_random_qkv, sweep_workload
+from tests.gpu_helpers import (assert_linear_states_close, assert_output_close,
+                               assert_prepare_bitexact, compare_lists, f32, run_gpu)
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_check(q, k, v, rho, nu, repeat=2):
+    g = run_gpu(q, k, v, rho, nu, repeat=repeat)
+    qf, kf, vf = f32(q), f32(k), f32(v)
+    prep = O.prepare(qf, kf)
+    sel = O.select(prep.q_bar, prep.k_bar, rho, nu)
+    assert_prepare_bitexact(g, prep)
+    assert (g["k_c"], g["n_neg"], g["m"]) == (sel.k_c, sel.n_neg, sel.m)
+    near = compare_lists(g, sel)
+    assert near == 0
+    B, H, N, _ = q.shape
+    assert_linear_states_close(g, prep, vf, [(0, 0), (B - 1, H - 1)], N)
+    ref = O.forward(prep, vf, sel)
+    unq = O.forward(prep, vf, sel, quant=False)
+    res = assert_output_close(g["out"], ref, unq)
+    for o in g["outs"][1:]:  # deterministic run to run
+        np.testing.assert_array_equal(o, g["outs"][0])
+    return g, res
+
+
+def test_tiny_workload():
+    wl = WORKLOADS["tiny"]
+    q, k, v = make_qkv(wl.B, wl.H, wl.grid, seed=0)
+    _full_check(q, k, v, wl.rho, wl.nu)
+
+
+def test_dense_workload_sageattention_only():
+    wl = WORKLOADS["dense"]
+    q, k, v = make_qkv(wl.B, wl.H, wl.grid, seed=0)
+    g, res = _full_check(q, k, v, wl.rho, wl.nu)
+    assert g["m"] == 0
+    # against fp64 full softmax attention of the bf16 inputs
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.double(), k.double(), v.double(), scale=float(O.softmax_scale(128))).numpy()
+    from tests.gpu_helpers import cos
+    assert cos(g["out"], ref) >= 0.99
+
+
+@pytest.mark.parametrize("N,rho,nu", [
+    (64, 1.0, 0.0),      # a single block
+    (65, 0.5, 0.0),      # two blocks, the second holds one token
+    (100, 0.5, 0.5),     # ragged, no marginal blocks (m = 0), one negligible
+    (191, 0.34, 0.33),   # odd number of blocks: the last CTA has one query block
+    (1000, 0.25, 0.25),  # ragged tail, marginal branch on
+    (2000, 0.1, 0.45),   # 480p-like ratios at a small size
+    (4096, 1.0, 0.0),
+])
+def test_edge_shapes(N, rho, nu):
+    q, k, v = make_random_qkv(1, 3, N, seed=N)
+    _full_check(q, k, v, rho, nu)
+
+
+def test_degenerate_blocks():
+    # an all-zero Q block (s_q = 0), a K block equal to its channel mean (K~ = 0 -> s_k may
+    # be tiny), identical key blocks (all logits tied) and a large outlier channel in K.
+    q, k, v = make_random_qkv(1, 2, 640, seed=3)
+    q[0, 0, 64:128] = 0
+    k[0, 1] = k[0, 1, :64].repeat(10, 1)
+    k[0, 0, :, 5] += 40.0
+    _full_check(q, k, v, 0.3, 0.3)
+
+
+def test_batch_two_sweep_shape_small():
+    wl = sweep_workload(0.2)
+    q, k, v = make_qkv(2, 2, (3, 16, 32), seed=1)
+    _full_check(q, k, v, wl.rho, wl.nu)
+
+
+def _sampled_check(wl, heads_for_oracle, qblocks_per_head, seed=0):
+    q, k, v = make_qkv(wl.B, wl.H, wl.grid, seed=seed)
+    g = run_gpu(q, k, v, wl.rho, wl.nu, repeat=1)
+    B, H, N, _ = q.shape
+    nB = -(-N // 64)
+    hs = slice(0, heads_for_oracle)
+    qf, kf, vf = f32(q[:, hs]), f32(k[:, hs]), f32(v[:, hs])
+    prep = O.prepare(qf, kf)
+    sel = O.select(prep.q_bar, prep.k_bar, wl.rho, wl.nu)
+    assert_prepare_bitexact(g, prep, hs)
+    near = compare_lists(g, sel, hs)
+    rng = np.random.default_rng(7)
+    qb = sorted(set(rng.choice(nB, size=qblocks_per_head, replace=False).tolist()) | {0, nB - 1})
+    heads = [(b, h) for b in range(B) for h in range(heads_for_oracle)]
+    ref = O.forward(prep, vf, sel, heads=heads, qblocks=qb)
+    unq = O.forward(prep, vf, sel, heads=heads, qblocks=qb, quant=False)
+    res = assert_output_close(g["out"][:, hs], ref, unq)
+    return near, res
+
+
+def test_480p_full_size_sampled():
+    near, res = _sampled_check(WORKLOADS["480p"], heads_for_oracle=3, qblocks_per_head=24)
+    assert near == 0
+
+
+def test_720p_full_size_sampled():
+    near, res = _sampled_check(WORKLOADS["720p"], heads_for_oracle=2, qblocks_per_head=12)
+    assert near == 0
+
+
+@pytest.mark.parametrize("rho", [1.0, 0.05])
+def test_sweep_full_size_sampled(rho):
+    near, res = _sampled_check(sweep_workload(rho), heads_for_oracle=1, qblocks_per_head=8, seed=1)
+    assert near == 0
