@@ -94,6 +94,23 @@ int sagesla_prepare(const sagesla_shape* shape, const void* q, const void* k,
                     float* k_bar, void* h, float* z, void* workspace,
                     size_t workspace_bytes, void* stream);
 
+/* sagesla_prepare for callers that cannot allocate device memory when they call it (an
+ * engine that owns every buffer from start-up, a plugin host, a loop that must not call
+ * cudaMalloc because it can synchronize the device). The paper has no counterpart: this
+ * is an interface variant, not a step of the method.
+ * Same inputs and outputs as sagesla_prepare, without a workspace: its scratch (the
+ * per-block channel sums of K and the status word) lives in a 24 MiB + 256 B __device__
+ * array inside the library, held on every GPU that loads the library until exit.
+ * Shapes needing more (B*H*ceil(N/64)*512 + 256 bytes) return SAGESLA_ERR_UNSUPPORTED
+ * before any launch. The first call on a device looks up the array's address with
+ * cudaGetSymbolAddress and should come before any stream capture. All calls share the
+ * array: calls whose kernels overlap on the GPU race on it (order them on one stream).
+ * Nothing is allocated; a timed-out device wait is not reported by this variant. */
+int sagesla_prepare_static_scratch(const sagesla_shape* shape, const void* q, const void* k,
+                                   const void* v, float sm_scale, int8_t* q8, int8_t* k8,
+                                   float* q_scale, float* k_scale, float* k_mean, float* q_bar,
+                                   float* k_bar, void* h, float* z, void* stream);
+
 /* Step (4): block logits, ranking and the per-row block lists.
  * Inputs : q_bar, k_bar fp32 [B,H,nB,d]; rho, nu as in sagesla_counts.
  * Outputs: crit_idx int32 [B,H,nB,k_c]  ascending critical key blocks per row

@@ -54,6 +54,8 @@ def lib():
     L.sagesla_reset_status.restype = ctypes.c_int
     L.sagesla_prepare.argtypes = [sp, _vp, _vp, _vp, ctypes.c_float] + [_vp] * 9 + [_vp, ctypes.c_size_t, _vp]
     L.sagesla_prepare.restype = ctypes.c_int
+    L.sagesla_prepare_static_scratch.argtypes = [sp, _vp, _vp, _vp, ctypes.c_float] + [_vp] * 9 + [_vp]
+    L.sagesla_prepare_static_scratch.restype = ctypes.c_int
     L.sagesla_select.argtypes = [sp, _vp, _vp, ctypes.c_double, ctypes.c_double, _vp, _vp, _vp, _vp, _vp]
     L.sagesla_select.restype = ctypes.c_int
     L.sagesla_forward.argtypes = ([sp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int,
@@ -165,6 +167,24 @@ def sagesla_prepare(q, k, v, workspace, sm_scale=None, out: Prepared | None = No
                                  _ptr(out.k8), _ptr(out.q_scale), _ptr(out.k_scale), _ptr(out.k_mean),
                                  _ptr(out.q_bar), _ptr(out.k_bar), _ptr(out.h), _ptr(out.z),
                                  _ptr(workspace), workspace.numel(), _stream(stream)), "sagesla_prepare")
+    return out
+
+
+def sagesla_prepare_static_scratch(q, k, v, sm_scale=None, out: Prepared | None = None, stream=None):
+    """sagesla_prepare without a workspace: the library keeps the small scratch this step
+    needs in its own fixed-size device array, for callers that cannot allocate here.
+    Calls share that array, so order them on one stream."""
+    B, H, N, d, nB = _dims(q)
+    for t in (q, k, v):
+        assert t.dtype == torch.bfloat16 and t.is_cuda and t.is_contiguous() and t.shape == q.shape
+    if out is None:
+        out = alloc_prepared(B, H, N, q.device)
+    c_s = softmax_scale(d) if sm_scale is None else float(sm_scale)
+    sh = _shape(B, H, N, d)
+    _check(lib().sagesla_prepare_static_scratch(
+        ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), c_s, _ptr(out.q8), _ptr(out.k8),
+        _ptr(out.q_scale), _ptr(out.k_scale), _ptr(out.k_mean), _ptr(out.q_bar), _ptr(out.k_bar),
+        _ptr(out.h), _ptr(out.z), _stream(stream)), "sagesla_prepare_static_scratch")
     return out
 
 
