@@ -29,17 +29,25 @@
 namespace sgs {
 namespace {
 
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kStageBytes = 8192 + 16384;  // K8 tile + V tile
 constexpr int kOffQ = 0;
 constexpr int kOffStage = 16384;
-constexpr int kOffP = kOffStage + kStages * kStageBytes;
-constexpr int kOffBar = kOffP + 2 * 16384;
-constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 2 + 1;
-constexpr int kAttnSmem = kOffBar + kNumBars * 8 + 16 + 1024;
+constexpr int kOffBar = kOffStage + kStages * kStageBytes;
+constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;
+constexpr int kAttnSmem = kOffBar + kNumBars * 8 + 16 + 1024;  // ~91 KB: two CTAs per SM
 constexpr int kAttnThreads = 192;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
+// Columns [0, kPolyCols) of every 64-key tile take exp2 on the FMA pipe (exp2_poly), the
+// rest on the SFU (ex2.approx): this balances the two pipes, the SFU alone being slower
+// than the tensor core at one exponential per score.
+constexpr int kPolyCols = 16;
+
+// TMEM columns: S0 [0,64), S1 [64,128) (int32 scores of one 128x64 tile; after the
+// softmax, columns [0,32) of S_b hold the bf16 P tile, two values per column), O [128,256).
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColO = 128;
 
 struct AttnParams {
   const float* q_scale;
@@ -67,14 +75,74 @@ struct UnionWalk {
   }
 };
 
-// A drain wait ignores the abort flag: it is used to let copies / MMAs already in flight
-// land before the CTA releases its shared memory and TMEM.
+// A drain wait ignores the abort flag: it lets copies / MMAs already in flight land
+// before the CTA releases its shared memory and TMEM.
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, int* status) {
   int never = 0;
   mbar_wait(bar, parity, &never, status);
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 1)
+// 2^x on the FMA pipe, for x <= ~9 (scores minus the running max, in log2 units).
+// Cody-Waite style range reduction x = n + f, n = rint(x), f in [-1/2, 1/2], then a
+// degree-3 polynomial for 2^f fitted for minimum relative error on [-1/2, 1/2]
+// (max relative error 7.5e-5, far below the bf16 rounding P receives), and 2^n added
+// to the exponent field. x is clamped at -125 so the exponent stays normal; 2^-125 is
+// negligible next to a row sum >= 1.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = __fadd_rn(x, 12582912.f);  // 1.5*2^23 + rint(x): rint in the low bits
+  const float n = __fsub_rn(t, 12582912.f);
+  const float f = __fsub_rn(x, n);
+  float p = fmaf(0.0551716648042202f, f, 0.2426111400127411f);
+  p = fmaf(p, f, 0.6932609677314758f);
+  p = fmaf(p, f, 0.9999280571937561f);
+  // (bits(t) << 23) == n << 23 (mod 2^32): the constant's low 9 bits are zero.
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Exact int32 -> fp32 for |v| < 2^22 (an INT8 dot product over 128 channels is at most
+// 128*127^2 < 2^21): add the bits of 1.5*2^23, subtract 1.5*2^23 as a float.
+__device__ __forceinline__ float i2f_exact(uint32_t v) {
+  return __fsub_rn(__int_as_float(static_cast<int>(v) + 0x4B400000), 12582912.f);
+}
+
+// One 64-key tile of one row: P = 2^(s*sc - m) rounded to bf16 pairs in pk, returns the
+// fp32 row sum of P. RAGGED masks columns >= nvalid to 0.
+template <bool RAGGED>
+__device__ __forceinline__ float softmax_tile(const uint32_t (&sv)[64], float sc, float negm,
+                                              int nvalid, uint32_t (&pk)[32]) {
+  float ps = 0.f;
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    const float x0 = fmaf(i2f_exact(sv[c]), sc, negm);
+    const float x1 = fmaf(i2f_exact(sv[c + 1]), sc, negm);
+    float p0 = c < kPolyCols ? exp2_poly(x0) : ex2_approx(x0);
+    float p1 = c + 1 < kPolyCols ? exp2_poly(x1) : ex2_approx(x1);
+    if (RAGGED) {
+      p0 = c < nvalid ? p0 : 0.f;
+      p1 = c + 1 < nvalid ? p1 : 0.f;
+    }
+    ps += p0 + p1;
+    pk[c >> 1] = pack_bf16x2(p0, p1);
+  }
+  return ps;
+}
+
+__device__ __forceinline__ void tmem_st32_sync(uint32_t taddr, const uint32_t (&r)[32]) {
+  tmem_st32(taddr, r);
+  tmem_wait_st();
+}
+
+// tcgen05.mma kind::f16 with the A operand (P, M x K) read from TMEM.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 2)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, AttnParams p) {
   extern __shared__ unsigned char smem_raw[];
@@ -85,8 +153,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* kv_full = q_full + 1;
   uint64_t* kv_empty = kv_full + kStages;
   uint64_t* s_full = kv_empty + kStages;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
+  uint64_t* p_full = s_full + 2;
   uint64_t* pv_done = p_full + 2;
   uint64_t* o_full = pv_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
@@ -114,7 +181,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(s_full + b), 1);
-      mbar_init(smem_u32(s_free + b), 128);
       mbar_init(smem_u32(p_full + b), 128);
       mbar_init(smem_u32(pv_done + b), 1);
     }
@@ -124,14 +190,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
   }
-  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 256);
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t taddr = *tmem_slot;
   const uint32_t sQ = smem_u32(smem + kOffQ);
   const uint32_t sStage = smem_u32(smem + kOffStage);
-  const uint32_t sP = smem_u32(smem + kOffP);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -163,6 +228,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Issue order QK(0), QK(1), PV(0), QK(2), PV(1), ...: tcgen05.mma ops from one thread
+    // execute in issue order, so QK(t) overwriting S_(t%2) (which holds P(t-2)) runs after
+    // PV(t-2) has read it.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = make_idesc(2, 1, 0, 0, 128, 64);
       constexpr uint32_t idesc_pv = make_idesc(1, 1, 0, 1, 128, 128);
@@ -174,8 +242,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t v = sStage + s * kStageBytes + 8192;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(taddr + 128, make_sdesc(sP + b * 16384 + kk * 32, 16, 1024),
-                   make_sdesc(v + kk * 2048, 8192, 1024), idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(taddr + kColO, taddr + 64 * b + 8 * kk, make_sdesc(v + kk * 2048, 8192, 1024),
+                      idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
         mma_commit(smem_u32(kv_empty + s));
         mma_commit(smem_u32(pv_done + b));
         return true;
@@ -184,10 +252,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       while (ok && walk.next(j, fl)) {
         const int s = t % kStages, b = t & 1;
         if (!mbar_wait(smem_u32(kv_full + s), (t / kStages) & 1, &abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        if (t >= 2 && !mbar_wait(smem_u32(s_free + b), ((t - 2) >> 1) & 1, &abort_flag, p.status)) {
           ok = false;
           break;
         }
@@ -210,6 +274,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax (warps 2-5)
+    // Thread = query row r of the 128-row tile; rows 0-63 are block i0, 64-127 block i0+1,
+    // so membership of a key block is uniform within each warp.
     const int wq = warp & 3;
     const int r = 32 * wq + lane;
     const int half = r >> 6;
@@ -224,82 +290,58 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int t = 0, j, fl;
     while (walk.next(j, fl)) {
       const int b = t & 1;
-      const bool member = (fl >> half) & 1;
+      const bool member = (fl >> half) & 1;  // warp-uniform
+      const float skj = sk[j];
       ok = mbar_wait(smem_u32(s_full + b), (t >> 1) & 1, &abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sv[64];
-      tmem_ld64_sync(taddr + lane_off + 64 * b, sv);
-      tc_fence_before();
-      mbar_arrive(smem_u32(s_free + b));
-      if (t >= 2) ok = mbar_wait(smem_u32(pv_done + b), ((t - 2) >> 1) & 1, &abort_flag, p.status);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
-      }
-
-      const int nvalid = (j == nB - 1) ? (p.N - j * 64) : 64;
-      float sc = 0.f, mt = -INFINITY;
+      uint32_t pk[32];
       if (member) {
-        int mx = INT_MIN;
+        uint32_t sv[64];
+        tmem_ld64_sync(taddr + lane_off + 64 * b, sv);
+        const bool ragged = (j == nB - 1) && (p.N - j * 64 < 64);  // CTA-uniform
+        const int nvalid = ragged ? p.N - j * 64 : 64;
+        int mx = static_cast<int>(sv[0]);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          if (c < nvalid) mx = max(mx, static_cast<int>(sv[c]));
-          if (c + 32 < nvalid) mx = max(mx, static_cast<int>(sv[c + 32]));
-        }
-        sc = __fmul_rn(__fmul_rn(sq, sk[j]), kLog2e);
-        mt = __fmul_rn(static_cast<float>(mx), sc);
-      }
-      const bool raise = member && (mt > m_run + kRescaleThreshold);
-      const bool resc = raise && (m_run != -INFINITY);
-      if (__any_sync(0xffffffffu, resc)) {
-        // O holds P.V of earlier tiles: wait for the last issued P.V, then rescale in TMEM.
-        if (t >= 1 &&
-            !mbar_wait(smem_u32(pv_done + ((t - 1) & 1)), ((t - 1) >> 1) & 1, &abort_flag, p.status)) {
-          ok = false;
-        }
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        const float alpha = resc ? ex2_approx(m_run - mt) : 1.f;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t o[32];
-          tmem_ld32_sync(taddr + lane_off + 128 + 32 * cc, o);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-          tmem_st32(taddr + lane_off + 128 + 32 * cc, o);
-        }
-        tmem_wait_st();
-        if (resc) l *= alpha;
-      }
-      if (raise) m_run = mt;
-
-      const uint32_t prow = sP + b * 16384;
-      float psum = 0.f;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float v0 = 0.f, v1 = 0.f;
-          const int c0 = 8 * q + 2 * e;
-          if (member) {
-            const uint32_t a0 = sv[c0];
-            const uint32_t a1 = sv[c0 + 1];
-            if (c0 < nvalid) v0 = ex2_approx(fmaf(static_cast<float>(static_cast<int>(a0)), sc, -m_run));
-            if (c0 + 1 < nvalid) v1 = ex2_approx(fmaf(static_cast<float>(static_cast<int>(a1)), sc, -m_run));
-            psum += v0 + v1;
+        for (int c = 1; c < 64; ++c)
+          if (!ragged || c < nvalid) mx = max(mx, static_cast<int>(sv[c]));
+        const float sc = __fmul_rn(__fmul_rn(sq, skj), kLog2e);
+        const float mt = __fmul_rn(static_cast<float>(mx), sc);
+        const bool raise = mt > m_run + kRescaleThreshold;
+        const bool resc = raise && (m_run != -INFINITY);
+        if (__any_sync(0xffffffffu, resc)) {
+          // O holds P.V of earlier tiles: wait for the last issued P.V, then rescale it.
+          if (t >= 1)
+            ok = mbar_wait(smem_u32(pv_done + ((t - 1) & 1)), ((t - 1) >> 1) & 1, &abort_flag,
+                           p.status);
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
           }
-          w[e] = pack_bf16x2(v0, v1);
+          tc_fence_after();
+          const float alpha = resc ? ex2_approx(m_run - mt) : 1.f;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t o[32];
+            tmem_ld32_sync(taddr + lane_off + kColO + 32 * cc, o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st32(taddr + lane_off + kColO + 32 * cc, o);
+          }
+          tmem_wait_st();
+          if (resc) l *= alpha;
         }
-        st_shared_v4(prow + sw128_offset(r, q), w[0], w[1], w[2], w[3]);
+        if (raise) m_run = mt;
+        l += ragged ? softmax_tile<true>(sv, sc, -m_run, nvalid, pk)
+                    : softmax_tile<false>(sv, sc, -m_run, 64, pk);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
-      l += psum;
-      fence_async_smem();
+      tmem_st32_sync(taddr + lane_off + 64 * b, pk);
       tc_fence_before();
       mbar_arrive(smem_u32(p_full + b));
       ++t;
@@ -317,7 +359,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t o[32];
-        tmem_ld32_sync(taddr + lane_off + 128 + 32 * cc, o);
+        tmem_ld32_sync(taddr + lane_off + kColO + 32 * cc, o);
         if (row_valid) {
           float lin[32];
 #pragma unroll
@@ -341,7 +383,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int qq = 0; qq < 4; ++qq) {
             float f[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(o[8 * qq + e]) * inv + lin[8 * qq + e];
+            for (int e = 0; e < 8; ++e) f[e] = fmaf(__uint_as_float(o[8 * qq + e]), inv, lin[8 * qq + e]);
             d4[qq] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
                                 pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
           }
@@ -351,7 +393,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(taddr, 256);
+  if (warp == 1) tmem_dealloc(taddr, kTmemCols);
 }
 
 }  // namespace

@@ -35,14 +35,26 @@ __global__ void __launch_bounds__(64) ksum_block_kernel(const __nv_bfloat16* __r
   dst[t] = make_float2(a0, a1);
 }
 
-__global__ void __launch_bounds__(128) kmean_kernel(const float* __restrict__ part,
+// mu[c] = (P_0[c] + P_1[c] + ... + P_{nB-1}[c]) / N, summed in block order. One CTA per
+// (head, 16-channel group): the partial sums are staged through shared memory in chunks of
+// 256 blocks so the sequential adds do not wait on global-memory latency.
+constexpr int kMeanChunk = 256;
+__global__ void __launch_bounds__(256) kmean_kernel(const float* __restrict__ part,
                                                     float* __restrict__ mu, int N, int nB) {
-  const int bh = blockIdx.x, c = threadIdx.x;
-  const float* src = part + static_cast<size_t>(bh) * nB * kHeadDim + c;
+  __shared__ float buf[kMeanChunk][17];
+  const int bh = blockIdx.x, c0 = 16 * blockIdx.y, tid = threadIdx.x;
+  const float* src = part + static_cast<size_t>(bh) * nB * kHeadDim + c0;
   float T = 0.f;
-#pragma unroll 8
-  for (int j = 0; j < nB; ++j) T = __fadd_rn(T, src[static_cast<size_t>(j) * kHeadDim]);
-  mu[bh * kHeadDim + c] = __fdiv_rn(T, static_cast<float>(N));
+  for (int base = 0; base < nB; base += kMeanChunk) {
+    const int n = min(kMeanChunk, nB - base);
+    for (int x = tid; x < n * 16; x += 256)
+      buf[x >> 4][x & 15] = src[static_cast<size_t>(base + (x >> 4)) * kHeadDim + (x & 15)];
+    __syncthreads();
+    if (tid < 16)
+      for (int jj = 0; jj < n; ++jj) T = __fadd_rn(T, buf[jj][tid]);
+    __syncthreads();
+  }
+  if (tid < 16) mu[bh * kHeadDim + c0 + tid] = __fdiv_rn(T, static_cast<float>(N));
 }
 
 struct PrepParams {
@@ -288,7 +300,7 @@ cudaError_t launch_prepare(const Dims& g, const void* q, const void* k, const vo
   }
   {
     TraceScope ts_("kmean_kernel", st);
-    kmean_kernel<<<g.BH, 128, 0, st>>>(part, k_mean, g.N, g.nB);
+    kmean_kernel<<<dim3(g.BH, kHeadDim / 16), 256, 0, st>>>(part, k_mean, g.N, g.nB);
   }
   cudaError_t e = cudaFuncSetAttribute(prep_block_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem);

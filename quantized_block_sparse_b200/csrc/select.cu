@@ -89,17 +89,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelParams p) {
   }
   __syncthreads();
 
-  // ---- 2. bitonic sort, descending, every row at once
+  // ---- 2. bitonic sort, descending, every row at once (nBpow = 2^lgn)
+  const int lgn = __ffs(nBpow) - 1;
   const int half = nBpow >> 1;
-  for (int k = 2; k <= nBpow; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+  for (int lk = 1; lk <= lgn; ++lk) {
+    for (int lj = lk - 1; lj >= 0; --lj) {
+      const int jj = 1 << lj;
       for (int x = tid; x < rows * half; x += kSelThreads) {
-        const int r = x / half, t = x - r * half;
-        const int i = (t / jj) * 2 * jj + (t % jj);
+        const int r = x >> (lgn - 1), t = x & (half - 1);
+        const int i = ((t >> lj) << (lj + 1)) | (t & (jj - 1));
         const int l = i + jj;
         uint64_t* kr = keys + r * nBpow;
         const uint64_t a = kr[i], b = kr[l];
-        const bool desc = (i & k) == 0;
+        const bool desc = ((i >> lk) & 1) == 0;
         if (desc ? (a < b) : (a > b)) {
           kr[i] = b;
           kr[l] = a;
@@ -110,10 +112,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelParams p) {
   }
 
   // ---- 3. classes by sorted position, then ascending compaction
-  for (int x = tid; x < rows * nB; x += kSelThreads) {
-    const int r = x / nB, pos = x - r * nB;
-    const int j = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(keys[r * nBpow + pos]));
-    cls[r * nBpow + j] = pos < p.k_c ? 0 : (pos < nB - p.n_neg ? 1 : 2);
+  for (int r = 0; r < rows; ++r) {
+    for (int pos = tid; pos < nB; pos += kSelThreads) {
+      const int j = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(keys[r * nBpow + pos]));
+      cls[r * nBpow + j] = pos < p.k_c ? 0 : (pos < nB - p.n_neg ? 1 : 2);
+    }
   }
   __syncthreads();
 
