@@ -34,15 +34,27 @@ constexpr int kStageBytes = 8192 + 16384;  // K8 tile + V tile
 constexpr int kOffQ = 0;
 constexpr int kOffStage = 16384;
 constexpr int kOffBar = kOffStage + kStages * kStageBytes;
-constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;
-constexpr int kAttnSmem = kOffBar + kNumBars * 8 + 16 + 1024;  // ~91 KB: two CTAs per SM
-constexpr int kAttnThreads = 192;
+constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1 + 1;
+constexpr int kOffMeta = kOffBar + 256;              // per-stage tile metadata (StageMeta)
+constexpr int kOffRowSum = kOffMeta + kStages * 16;  // final row sums, [128]
+constexpr int kAttnSmem = kOffRowSum + 128 * 4 + 1024;  // ~91 KB: two CTAs per SM
+constexpr int kSoftmaxWarps = 8;
+constexpr int kAttnThreads = 64 + 32 * kSoftmaxWarps;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
-// Columns [0, kPolyCols) of every 64-key tile take exp2 on the FMA pipe (exp2_poly), the
-// rest on the SFU (ex2.approx): this balances the two pipes, the SFU alone being slower
-// than the tensor core at one exponential per score.
-constexpr int kPolyCols = 16;
+// Of every 64-key tile a softmax thread holds 2 rows x 16 keys, in 8 groups ("reps") of
+// 2 keys per row; the first kPolyReps groups take exp2 on the FMA pipe (exp2_poly2), the rest
+// on the SFU (ex2.approx). Raising it moves exponentials off the SFU when that is the limit.
+constexpr int kPolyReps = 0;
+
+// Written by the TMA producer for every union step, read by the MMA issuer and the softmax
+// warps after they observe the stage's kv_full phase (mbarrier release/acquire).
+struct StageMeta {
+  int j;       // key block
+  int flags;   // bit 0: critical for query block i0, bit 1: for i0+1, bit 2: last step
+  float sk;    // k_scale of block j
+  int pad;
+};
 
 // TMEM columns: S0 [0,64), S1 [64,128) (int32 scores of one 128x64 tile; after the
 // softmax, columns [0,32) of S_b hold the bf16 P tile, two values per column), O [128,256).
@@ -82,50 +94,149 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, int* s
   mbar_wait(bar, parity, &never, status);
 }
 
-// 2^x on the FMA pipe, for x <= ~9 (scores minus the running max, in log2 units).
+// ---- packed fp32 pairs (Blackwell f32x2 FMA / add: two lanes per instruction)
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
+constexpr int kMagicBits = 0x4B400000;
+
+// 2^x on the FMA pipe for two values, x <= ~9 (scores minus the running max, log2 units).
 // Cody-Waite style range reduction x = n + f, n = rint(x), f in [-1/2, 1/2], then a
-// degree-3 polynomial for 2^f fitted for minimum relative error on [-1/2, 1/2]
-// (max relative error 7.5e-5, far below the bf16 rounding P receives), and 2^n added
-// to the exponent field. x is clamped at -125 so the exponent stays normal; 2^-125 is
-// negligible next to a row sum >= 1.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = __fadd_rn(x, 12582912.f);  // 1.5*2^23 + rint(x): rint in the low bits
-  const float n = __fsub_rn(t, 12582912.f);
-  const float f = __fsub_rn(x, n);
-  float p = fmaf(0.0551716648042202f, f, 0.2426111400127411f);
-  p = fmaf(p, f, 0.6932609677314758f);
-  p = fmaf(p, f, 0.9999280571937561f);
-  // (bits(t) << 23) == n << 23 (mod 2^32): the constant's low 9 bits are zero.
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+// degree-3 polynomial for 2^f fitted for minimum relative error on [-1/2, 1/2] (max
+// relative error 7.5e-5, far below the bf16 rounding P receives), and n added to the
+// exponent field. x is clamped at -125 so the exponent stays normal; 2^-125 is negligible
+// next to a row sum >= 1.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  const uint64_t x = f2pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = add2(x, f2pack(kMagic, kMagic));      // 1.5*2^23 + rint(x)
+  const uint64_t n = add2(t, f2pack(-kMagic, -kMagic));    // rint(x), exact
+  const uint64_t f = fma2(n, f2pack(-1.f, -1.f), x);       // x - rint(x), exact
+  uint64_t p = fma2(f2pack(0.0551716648042202f, 0.0551716648042202f), f,
+                    f2pack(0.2426111400127411f, 0.2426111400127411f));
+  p = fma2(p, f, f2pack(0.6932609677314758f, 0.6932609677314758f));
+  p = fma2(p, f, f2pack(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, t0, t1;
+  f2unpack(p, p0, p1);
+  f2unpack(t, t0, t1);
+  // (bits(t) << 23) == rint(x) << 23 (mod 2^32): the constant's low 9 bits are zero.
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
-// Exact int32 -> fp32 for |v| < 2^22 (an INT8 dot product over 128 channels is at most
-// 128*127^2 < 2^21): add the bits of 1.5*2^23, subtract 1.5*2^23 as a float.
-__device__ __forceinline__ float i2f_exact(uint32_t v) {
-  return __fsub_rn(__int_as_float(static_cast<int>(v) + 0x4B400000), 12582912.f);
+// ---- TMEM access in the 16-lane shapes. For a 16-lane group starting at TMEM lane LB,
+// thread t of the warp holds rows LB + t/4 and LB + t/4 + 8:
+//   16x256b (8 columns per repetition k): regs 4k..4k+3 = (row0, 8k+2q), (row0, 8k+2q+1),
+//           (row1, 8k+2q), (row1, 8k+2q+1) with q = t%4;
+//   16x128b (4 columns per repetition k): regs 2k, 2k+1 = (row0, 4k+q), (row1, 4k+q).
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_16x128b_x8(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
 }
 
-// One 64-key tile of one row: P = 2^(s*sc - m) rounded to bf16 pairs in pk, returns the
-// fp32 row sum of P. RAGGED masks columns >= nvalid to 0.
+// The softmax of one thread's share of a 64-key tile: rows row0/row1, 16 keys each (A: the
+// exact floats 1.5*2^23 + int32 score in the 16x256b register order; the INT8 dot product
+// over 128 channels is at most 128*127^2 < 2^22 in magnitude, so the integer is exact in the
+// mantissa). P = 2^((A - 1.5*2^23)*sc - m_row), rounded to bf16 pairs in pk (16x128b order);
+// returns the fp32 sums of this thread's P per row. Keys >= nvalid (a ragged last key block)
+// get P = 0.
 template <bool RAGGED>
-__device__ __forceinline__ float softmax_tile(const uint32_t (&sv)[64], float sc, float negm,
-                                              int nvalid, uint32_t (&pk)[32]) {
-  float ps = 0.f;
+__device__ __forceinline__ void softmax_tile(const float (&A)[32], float sc, float negm0,
+                                             float negm1, int q, int nvalid, uint32_t (&pk)[16],
+                                             float& ps0, float& ps1) {
+  const uint64_t sub = f2pack(-kMagic, -kMagic), sc2 = f2pack(sc, sc);
+  const uint64_t nm0 = f2pack(negm0, negm0), nm1 = f2pack(negm1, negm1);
+  uint64_t acc0 = 0ull, acc1 = 0ull;
 #pragma unroll
-  for (int c = 0; c < 64; c += 2) {
-    const float x0 = fmaf(i2f_exact(sv[c]), sc, negm);
-    const float x1 = fmaf(i2f_exact(sv[c + 1]), sc, negm);
-    float p0 = c < kPolyCols ? exp2_poly(x0) : ex2_approx(x0);
-    float p1 = c + 1 < kPolyCols ? exp2_poly(x1) : ex2_approx(x1);
-    if (RAGGED) {
-      p0 = c < nvalid ? p0 : 0.f;
-      p1 = c + 1 < nvalid ? p1 : 0.f;
+  for (int k = 0; k < 8; ++k) {
+    const uint64_t x0 = fma2(add2(f2pack(A[4 * k], A[4 * k + 1]), sub), sc2, nm0);
+    const uint64_t x1 = fma2(add2(f2pack(A[4 * k + 2], A[4 * k + 3]), sub), sc2, nm1);
+    float a0, a1, b0, b1, pa0, pa1, pb0, pb1;
+    f2unpack(x0, a0, a1);
+    f2unpack(x1, b0, b1);
+    if (k < kPolyReps) {
+      exp2_poly2(a0, a1, pa0, pa1);
+      exp2_poly2(b0, b1, pb0, pb1);
+    } else {
+      pa0 = ex2_approx(a0);
+      pa1 = ex2_approx(a1);
+      pb0 = ex2_approx(b0);
+      pb1 = ex2_approx(b1);
     }
-    ps += p0 + p1;
-    pk[c >> 1] = pack_bf16x2(p0, p1);
+    if (RAGGED) {
+      const int c = 8 * k + 2 * q;
+      if (c >= nvalid) pa0 = pb0 = 0.f;
+      if (c + 1 >= nvalid) pa1 = pb1 = 0.f;
+    }
+    acc0 = add2(acc0, f2pack(pa0, pa1));
+    acc1 = add2(acc1, f2pack(pb0, pb1));
+    pk[2 * k] = pack_bf16x2(pa0, pa1);
+    pk[2 * k + 1] = pack_bf16x2(pb0, pb1);
   }
-  return ps;
+  float a, b, c, d;
+  f2unpack(acc0, a, b);
+  f2unpack(acc1, c, d);
+  ps0 = a + b;
+  ps1 = c + d;
+}
+
+__device__ __forceinline__ float quad_max(float v) {
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+}
+__device__ __forceinline__ float quad_sum(float v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  return v + __shfl_xor_sync(0xffffffffu, v, 2);
 }
 
 __device__ __forceinline__ void tmem_st32_sync(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -156,7 +267,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   uint64_t* p_full = s_full + 2;
   uint64_t* pv_done = p_full + 2;
   uint64_t* o_full = pv_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
+  uint64_t* lsum_bar = o_full + 1;  // final row sums written (all softmax threads)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lsum_bar + 1);
+  StageMeta* meta = reinterpret_cast<StageMeta*>(smem + kOffMeta);
+  float* rowsum = reinterpret_cast<float*>(smem + kOffRowSum);
   __shared__ int abort_flag;
 
   const int pr = blockIdx.x, bh = blockIdx.y;
@@ -181,10 +295,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(s_full + b), 1);
-      mbar_init(smem_u32(p_full + b), 128);
+      mbar_init(smem_u32(p_full + b), 32 * kSoftmaxWarps);
       mbar_init(smem_u32(pv_done + b), 1);
     }
     mbar_init(smem_u32(o_full), 1);
+    mbar_init(smem_u32(lsum_bar), 32 * kSoftmaxWarps);
     fence_mbar_init();
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
@@ -206,19 +321,28 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       tma_load_3d(sQ + 8192, &tmQ, smem_u32(q_full), 0, i0 * 64 + 64, bh);
       int t = 0, j, fl;
       bool aborted = false;
-      while (walk.next(j, fl)) {
+      bool have = walk.next(j, fl);  // k_c >= 1: at least one step
+      while (have) {
+        int jn, fln;
+        const bool have_next = walk.next(jn, fln);
         const int s = t % kStages;
         if (t >= kStages &&
             !mbar_wait(smem_u32(kv_empty + s), ((t / kStages) - 1) & 1, &abort_flag, p.status)) {
           aborted = true;
           break;
         }
+        meta[s].j = j;
+        meta[s].flags = fl | (have_next ? 0 : 4);
+        meta[s].sk = __ldg(p.k_scale + static_cast<size_t>(bh) * nB + j);
         const uint32_t dst = sStage + s * kStageBytes;
         mbar_expect_tx(smem_u32(kv_full + s), kStageBytes);
         tma_load_3d(dst, &tmK, smem_u32(kv_full + s), 0, j * 64, bh);
         tma_load_3d(dst + 8192, &tmV, smem_u32(kv_full + s), 0, j * 64, bh);
         tma_load_3d(dst + 16384, &tmV, smem_u32(kv_full + s), 64, j * 64, bh);
         ++t;
+        have = have_next;
+        j = jn;
+        fl = fln;
       }
       if (aborted || abort_flag) {  // let the copies in flight land before exit
         mbar_drain(smem_u32(q_full), 0, p.status);
@@ -248,13 +372,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         mma_commit(smem_u32(pv_done + b));
         return true;
       };
-      int t = 0, j, fl;
-      while (ok && walk.next(j, fl)) {
+      int t = 0;
+      bool last = false;
+      while (ok && !last) {
         const int s = t % kStages, b = t & 1;
         if (!mbar_wait(smem_u32(kv_full + s), (t / kStages) & 1, &abort_flag, p.status)) {
           ok = false;
           break;
         }
+        last = (meta[s].flags & 4) != 0;
         tc_fence_after();
         const uint32_t kt = sStage + s * kStageBytes;
 #pragma unroll
@@ -273,47 +399,99 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       mbar_drain(smem_u32(o_full), 0, p.status);
     }
   } else {
-    // ------------------------------------------------------------ softmax (warps 2-5)
-    // Thread = query row r of the 128-row tile; rows 0-63 are block i0, 64-127 block i0+1,
-    // so membership of a key block is uniform within each warp.
+    // ------------------------------------------------------------ softmax (warps 2-9)
+    // Warp w owns the 16 TMEM lanes LB = 32*(w%4) + 16*((w-2)/4) .. LB+15 (query rows of the
+    // 128-row tile); in the 16-lane load shape thread t holds rows LB + t/4 and LB + t/4 + 8,
+    // 16 keys each, and the four threads of a quad (t/4) share rows. Rows 0-63 are block i0,
+    // 64-127 block i0+1, so membership is warp-uniform.
     const int wq = warp & 3;
-    const int r = 32 * wq + lane;
-    const int half = r >> 6;
+    const int sub = (warp - 2) >> 2;
+    const uint32_t lb = 32 * wq + 16 * sub;
+    const int q = lane & 3;
+    const int rr0 = static_cast<int>(lb) + (lane >> 2);  // rows rr0 and rr0 + 8
+    const int half = rr0 >> 6;
     const int i = i0 + half;
-    const int tok = i * 64 + (r & 63);
-    const bool row_valid = (i < nB) && (tok < p.N);
     const float sq = (i < nB) ? p.q_scale[static_cast<size_t>(bh) * nB + i] : 0.f;
-    const float* sk = p.k_scale + static_cast<size_t>(bh) * nB;
-    const uint32_t lane_off = static_cast<uint32_t>(32 * wq) << 16;
-    float m_run = -INFINITY, l = 0.f;
+    const uint32_t lane_off = lb << 16;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     bool ok = true;
-    int t = 0, j, fl;
-    while (walk.next(j, fl)) {
-      const int b = t & 1;
-      const bool member = (fl >> half) & 1;  // warp-uniform
-      const float skj = sk[j];
+    bool last = false;
+    int t = 0;
+    while (!last) {
+      const int b = t & 1, s = t % kStages;
       ok = mbar_wait(smem_u32(s_full + b), (t >> 1) & 1, &abort_flag, p.status);
+      ok = ok && mbar_wait(smem_u32(kv_full + s), (t / kStages) & 1, &abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t pk[32];
+      const int j = meta[s].j, fl = meta[s].flags;
+      const float skj = meta[s].sk;
+      last = (fl & 4) != 0;
+      const bool member = (fl >> half) & 1;  // warp-uniform
+      uint32_t pk[16];
       if (member) {
-        uint32_t sv[64];
-        tmem_ld64_sync(taddr + lane_off + 64 * b, sv);
+        uint32_t sv[32];
+        tmem_ld_16x256b_x8(taddr + lane_off + 64 * b, sv);
         const bool ragged = (j == nB - 1) && (p.N - j * 64 < 64);  // CTA-uniform
         const int nvalid = ragged ? p.N - j * 64 : 64;
-        int mx = static_cast<int>(sv[0]);
+        float A[32];
 #pragma unroll
-        for (int c = 1; c < 64; ++c)
-          if (!ragged || c < nvalid) mx = max(mx, static_cast<int>(sv[c]));
+        for (int c = 0; c < 32; ++c) A[c] = __int_as_float(static_cast<int>(sv[c]) + kMagicBits);
+        float mA0 = 0.f, mA1 = 0.f;  // 0 is below every real value (all >= 1.5*2^23 - 2^22)
+        if (!ragged) {
+          mA0 = fmax3(A[0], A[1], A[4]);
+          mA1 = fmax3(A[2], A[3], A[6]);
+          mA0 = fmax3(mA0, A[5], A[8]);
+          mA1 = fmax3(mA1, A[7], A[10]);
+#pragma unroll
+          for (int k = 2; k < 8; ++k) {
+            if (k == 2) {
+              mA0 = fmax3(mA0, A[9], A[12]);
+              mA1 = fmax3(mA1, A[11], A[14]);
+            } else if (k < 7) {
+              mA0 = fmax3(mA0, A[4 * k + 1], A[4 * k + 4]);
+              mA1 = fmax3(mA1, A[4 * k + 3], A[4 * k + 6]);
+            } else {
+              mA0 = fmaxf(mA0, A[29]);
+              mA1 = fmaxf(mA1, A[31]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int c = 8 * k + 2 * q;
+            if (c < nvalid) {
+              mA0 = fmaxf(mA0, A[4 * k]);
+              mA1 = fmaxf(mA1, A[4 * k + 2]);
+            }
+            if (c + 1 < nvalid) {
+              mA0 = fmaxf(mA0, A[4 * k + 1]);
+              mA1 = fmaxf(mA1, A[4 * k + 3]);
+            }
+          }
+        }
+        mA0 = quad_max(mA0);
+        mA1 = quad_max(mA1);
         const float sc = __fmul_rn(__fmul_rn(sq, skj), kLog2e);
-        const float mt = __fmul_rn(static_cast<float>(mx), sc);
-        const bool raise = mt > m_run + kRescaleThreshold;
-        const bool resc = raise && (m_run != -INFINITY);
-        if (__any_sync(0xffffffffu, resc)) {
-          // O holds P.V of earlier tiles: wait for the last issued P.V, then rescale it.
+        const float mt0 = __fmul_rn(__fsub_rn(mA0, kMagic), sc);
+        const float mt1 = __fmul_rn(__fsub_rn(mA1, kMagic), sc);
+        const bool raise0 = mt0 > m0 + kRescaleThreshold, raise1 = mt1 > m1 + kRescaleThreshold;
+        const bool resc0 = raise0 && (m0 != -INFINITY), resc1 = raise1 && (m1 != -INFINITY);
+        const float alpha0 = resc0 ? ex2_approx(m0 - mt0) : 1.f;
+        const float alpha1 = resc1 ? ex2_approx(m1 - mt1) : 1.f;
+        if (raise0) m0 = mt0;
+        if (raise1) m1 = mt1;
+        float ps0, ps1;
+        if (ragged)
+          softmax_tile<true>(A, sc, -m0, -m1, q, nvalid, pk, ps0, ps1);
+        else
+          softmax_tile<false>(A, sc, -m0, -m1, q, 64, pk, ps0, ps1);
+        l0 = fmaf(l0, alpha0, ps0);
+        l1 = fmaf(l1, alpha1, ps1);
+        if (__any_sync(0xffffffffu, resc0 || resc1)) {
+          // O holds P.V of earlier tiles: wait for the last issued P.V, then rescale rows.
           if (t >= 1)
             ok = mbar_wait(smem_u32(pv_done + ((t - 1) & 1)), ((t - 1) >> 1) & 1, &abort_flag,
                            p.status);
@@ -322,44 +500,62 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             break;
           }
           tc_fence_after();
-          const float alpha = resc ? ex2_approx(m_run - mt) : 1.f;
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
+          for (int cc = 0; cc < 2; ++cc) {  // 2 x 64 columns of O (16x256b.x8 spans 64)
             uint32_t o[32];
-            tmem_ld32_sync(taddr + lane_off + kColO + 32 * cc, o);
+            const uint32_t oa = taddr + lane_off + kColO + 64 * cc;
+            tmem_ld_16x256b_x8(oa, o);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(taddr + lane_off + kColO + 32 * cc, o);
+            for (int k = 0; k < 8; ++k) {
+              o[4 * k] = __float_as_uint(__uint_as_float(o[4 * k]) * alpha0);
+              o[4 * k + 1] = __float_as_uint(__uint_as_float(o[4 * k + 1]) * alpha0);
+              o[4 * k + 2] = __float_as_uint(__uint_as_float(o[4 * k + 2]) * alpha1);
+              o[4 * k + 3] = __float_as_uint(__uint_as_float(o[4 * k + 3]) * alpha1);
+            }
+            tmem_st_16x256b_x8(oa, o);
           }
           tmem_wait_st();
-          if (resc) l *= alpha;
         }
-        if (raise) m_run = mt;
-        l += ragged ? softmax_tile<true>(sv, sc, -m_run, nvalid, pk)
-                    : softmax_tile<false>(sv, sc, -m_run, 64, pk);
       } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+        for (int c = 0; c < 16; ++c) pk[c] = 0u;
       }
-      tmem_st32_sync(taddr + lane_off + 64 * b, pk);
+      tmem_st_16x128b_x8(taddr + lane_off + 64 * b, pk);
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(p_full + b));
       ++t;
     }
 
     // ------------------------------------------------------------ epilogue
+    // Row sums: quad reduce, then hand them to the one-row-per-thread epilogue layout.
+    l0 = quad_sum(l0);
+    l1 = quad_sum(l1);
+    if (q == 0) {
+      rowsum[rr0] = l0;
+      rowsum[rr0 + 8] = l1;
+    }
+    mbar_arrive(smem_u32(lsum_bar));
+    ok = ok && mbar_wait(smem_u32(lsum_bar), 0, &abort_flag, p.status);
     ok = ok && mbar_wait(smem_u32(o_full), 0, &abort_flag, p.status);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
+    // Epilogue layout: warp w reads its quadrant's 32 lanes (32x32b), one row per thread,
+    // output columns [64*sub, 64*sub + 64).
+    const int r = 32 * wq + lane;
+    const int ie = i0 + (r >> 6);
+    const int tok = ie * 64 + (r & 63);
+    const bool row_valid = (ie < nB) && (tok < p.N);
+    const uint32_t eoff = static_cast<uint32_t>(32 * wq) << 16;
     if (ok) {
-      const float inv = 1.f / l;
-      const __nv_bfloat16* olr =
-          p.Ol ? p.Ol + (static_cast<size_t>(bh) * p.N + (row_valid ? tok : 0)) * kHeadDim : nullptr;
-      __nv_bfloat16* dst = p.out + (static_cast<size_t>(bh) * p.N + (row_valid ? tok : 0)) * kHeadDim;
+      const float inv = 1.f / rowsum[r];
+      const size_t row = static_cast<size_t>(bh) * p.N + (row_valid ? tok : 0);
+      const __nv_bfloat16* olr = p.Ol ? p.Ol + row * kHeadDim + 64 * sub : nullptr;
+      __nv_bfloat16* dst = p.out + row * kHeadDim + 64 * sub;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t o[32];
-        tmem_ld32_sync(taddr + lane_off + kColO + 32 * cc, o);
+        tmem_ld32_sync(taddr + eoff + kColO + 64 * sub + 32 * cc, o);
         if (row_valid) {
           float lin[32];
 #pragma unroll

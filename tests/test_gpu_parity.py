@@ -78,6 +78,23 @@ def test_degenerate_blocks():
     _full_check(q, k, v, 0.3, 0.3)
 
 
+def test_running_max_rises_every_tile():
+    # Scores grow with the key block index (K_j = (j+1) * u + noise, Q aligned with u), so
+    # the running row max rises by far more than 2^8 on every tile of the ascending walk and
+    # the O rescale path runs on every tile; with rho < 1 also on union tiles of one half.
+    g = torch.Generator().manual_seed(11)
+    N = 1100
+    u = torch.randn(128, generator=g, dtype=torch.float64)
+    u = u / u.norm() * 9.0
+    tok_blk = (torch.arange(N, dtype=torch.float64) // 64 + 1)[:, None]
+    k = tok_blk * u[None, :] + 0.3 * torch.randn(N, 128, generator=g, dtype=torch.float64)
+    q = u[None, :] + 0.3 * torch.randn(N, 128, generator=g, dtype=torch.float64)
+    v = torch.randn(N, 128, generator=g, dtype=torch.float64)
+    q, k, v = (x[None, None].repeat(1, 2, 1, 1).to(torch.bfloat16) for x in (q, k, v))
+    _full_check(q, k, v, 1.0, 0.0)
+    _full_check(q, k, v, 0.4, 0.2)
+
+
 def test_batch_two_sweep_shape_small():
     wl = sweep_workload(0.2)
     q, k, v = make_qkv(2, 2, (3, 16, 32), seed=1)
