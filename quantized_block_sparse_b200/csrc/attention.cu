@@ -29,26 +29,39 @@
 namespace sgs {
 namespace {
 
-constexpr int kStages = 3;
-constexpr int kStageBytes = 8192 + 16384;  // K8 tile + V tile
+// K tiles (8 KB, read only by QK^T) and V tiles (16 KB, read by P.V after the softmax) sit
+// in separate rings: a K slot frees as soon as its QK^T completes, so K runs far ahead;
+// a V slot frees when its P.V completes.
+constexpr int kKStages = 5;
+constexpr int kVStages = 3;
+constexpr int kKBytes = 8192;
+constexpr int kVBytes = 16384;
 constexpr int kOffQ = 0;
-constexpr int kOffStage = 16384;
-constexpr int kOffBar = kOffStage + kStages * kStageBytes;
-constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1 + 1;
-constexpr int kOffMeta = kOffBar + 256;              // per-stage tile metadata (StageMeta)
-constexpr int kOffRowSum = kOffMeta + kStages * 16;  // final row sums, [128]
-constexpr int kAttnSmem = kOffRowSum + 128 * 4 + 1024;  // ~91 KB: two CTAs per SM
+constexpr int kOffK = 16384;
+constexpr int kOffV = kOffK + kKStages * kKBytes;
+constexpr int kOffBar = kOffV + kVStages * kVBytes;
+constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 8 + 4 + 2 + 1 + 1;
+constexpr int kOffMeta = kOffBar + 512;               // per-K-slot tile metadata (StageMeta)
+constexpr int kOffRowSum = kOffMeta + kKStages * 16;  // final row sums, [128]
+constexpr int kAttnSmem = kOffRowSum + 128 * 4 + 1024;  // ~106 KB: two CTAs per SM
+static_assert(kNumBars * 8 + 4 <= kOffMeta - kOffBar, "barriers + TMEM slot overflow");
+static_assert(2 * (kAttnSmem + 1024) <= 233472, "two CTAs per SM must fit in shared memory");
 constexpr int kSoftmaxWarps = 8;
 constexpr int kAttnThreads = 64 + 32 * kSoftmaxWarps;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThreshold = 8.0f;
+// The softmax reference point m of a row is raised only when a thread's partial sum of
+// 2^(s - m) over its 16 keys of a tile exceeds 2^24 (or is not finite). Every accepted P is
+// then <= 2^24, the row sum l <= 2^41 and O stays far from fp32 overflow; the exact tile
+// max is computed only on that rare path (and on a row's first tile, where m = -inf).
+constexpr float kPsumLimit = 16777216.0f;
 // Of every 64-key tile a softmax thread holds 2 rows x 16 keys, in 8 groups ("reps") of
 // 2 keys per row; the first kPolyReps groups take exp2 on the FMA pipe (exp2_poly2), the rest
 // on the SFU (ex2.approx). Raising it moves exponentials off the SFU when that is the limit.
 constexpr int kPolyReps = 0;
 
-// Written by the TMA producer for every union step, read by the MMA issuer and the softmax
-// warps after they observe the stage's kv_full phase (mbarrier release/acquire).
+// Written by the TMA producer for every union step next to its K tile, read by the MMA
+// issuer and the softmax warps after they observe the slot's k_full phase (mbarrier
+// release/acquire).
 struct StageMeta {
   int j;       // key block
   int flags;   // bit 0: critical for query block i0, bit 1: for i0+1, bit 2: last step
@@ -234,6 +247,10 @@ __device__ __forceinline__ float quad_max(float v) {
   v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
   return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
 }
+__device__ __forceinline__ bool quad_any(bool v) {
+  const unsigned bal = __ballot_sync(0xffffffffu, v);
+  return ((bal >> ((threadIdx.x & 28u))) & 0xfu) != 0u;
+}
 __device__ __forceinline__ float quad_sum(float v) {
   v += __shfl_xor_sync(0xffffffffu, v, 1);
   return v + __shfl_xor_sync(0xffffffffu, v, 2);
@@ -253,6 +270,19 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
 }
 
+// Same, with the disable-output-lane mask: bit k of the 128-bit mask (m0 = lanes 0-31, ...,
+// m3 = lanes 96-127) keeps D lane k unchanged. Used for union steps that are critical for
+// only one of the two query blocks.
+__device__ __forceinline__ void mma_bf16_ts_masked(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                                   uint32_t idesc, uint32_t accumulate,
+                                                   uint32_t m0, uint32_t m1, uint32_t m2,
+                                                   uint32_t m3) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate), "r"(m0), "r"(m1), "r"(m2), "r"(m3));
+}
+
 __global__ void __launch_bounds__(kAttnThreads, 2)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, AttnParams p) {
@@ -261,11 +291,17 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = q_full + 1;
-  uint64_t* kv_empty = kv_full + kStages;
-  uint64_t* s_full = kv_empty + kStages;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 2;
+  uint64_t* k_full = q_full + 1;
+  uint64_t* k_empty = k_full + kKStages;
+  uint64_t* v_full = k_empty + kKStages;
+  uint64_t* v_empty = v_full + kVStages;
+  // S ready for step t: s_full[t % 8], phase parity (t / 8) & 1. Eight barriers (for two
+  // TMEM buffers) because a warp that skips steps (its half not critical) may reach step t
+  // as early as the completion of QK(t-5) (the K ring depth); the barrier's previous phase,
+  // step t-8, is then always complete, so a parity wait can never alias.
+  uint64_t* s_full = v_empty + kVStages;
+  uint64_t* p_full = s_full + 8;  // [half][buffer]
+  uint64_t* pv_done = p_full + 4;
   uint64_t* o_full = pv_done + 2;
   uint64_t* lsum_bar = o_full + 1;  // final row sums written (all softmax threads)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lsum_bar + 1);
@@ -289,13 +325,18 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   if (tid == 0) {
     abort_flag = 0;
     mbar_init(smem_u32(q_full), 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(kv_full + s), 1);
-      mbar_init(smem_u32(kv_empty + s), 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(smem_u32(k_full + s), 1);
+      mbar_init(smem_u32(k_empty + s), 1 + kSoftmaxWarps);  // QK commit + one per softmax warp
     }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(smem_u32(v_full + s), 1);
+      mbar_init(smem_u32(v_empty + s), 1);  // P.V commit
+    }
+    for (int x = 0; x < 8; ++x) mbar_init(smem_u32(s_full + x), 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(s_full + b), 1);
-      mbar_init(smem_u32(p_full + b), 32 * kSoftmaxWarps);
+      mbar_init(smem_u32(p_full + b), 128);      // half 0 rows, buffer b
+      mbar_init(smem_u32(p_full + 2 + b), 128);  // half 1 rows, buffer b
       mbar_init(smem_u32(pv_done + b), 1);
     }
     mbar_init(smem_u32(o_full), 1);
@@ -311,90 +352,162 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   tc_fence_after();
   const uint32_t taddr = *tmem_slot;
   const uint32_t sQ = smem_u32(smem + kOffQ);
-  const uint32_t sStage = smem_u32(smem + kOffStage);
+  const uint32_t sK = smem_u32(smem + kOffK);
+  const uint32_t sV = smem_u32(smem + kOffV);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // One thread feeds both rings without blocking on either: K tiles (with the step's
+    // metadata) run up to kKStages steps ahead of the V tiles.
     if (lane == 0) {
       mbar_expect_tx(smem_u32(q_full), 16384);
       tma_load_3d(sQ, &tmQ, smem_u32(q_full), 0, i0 * 64, bh);
       tma_load_3d(sQ + 8192, &tmQ, smem_u32(q_full), 0, i0 * 64 + 64, bh);
-      int t = 0, j, fl;
-      bool aborted = false;
+      int j, fl;
       bool have = walk.next(j, fl);  // k_c >= 1: at least one step
-      while (have) {
-        int jn, fln;
-        const bool have_next = walk.next(jn, fln);
-        const int s = t % kStages;
-        if (t >= kStages &&
-            !mbar_wait(smem_u32(kv_empty + s), ((t / kStages) - 1) & 1, &abort_flag, p.status)) {
+      int tK = 0, tV = 0, nsteps = -1;  // nsteps: known once the walk is exhausted
+      int ks = 0, kph = 0, vs = 0, vph = 0;
+      unsigned long long t_idle = 0;
+      bool aborted = false;
+      for (;;) {
+        bool progress = false;
+        // K: as far ahead as the ring allows (and never more than kKStages beyond V)
+        while (have && tK < tV + kKStages &&
+               (tK < kKStages || mbar_test_wait(smem_u32(k_empty + ks), kph ^ 1))) {
+          int jn, fln;
+          const bool have_next = walk.next(jn, fln);
+          meta[ks].j = j;
+          meta[ks].flags = fl | (have_next ? 0 : 4);
+          meta[ks].sk = __ldg(p.k_scale + static_cast<size_t>(bh) * nB + j);
+          mbar_expect_tx(smem_u32(k_full + ks), kKBytes);
+          tma_load_3d(sK + ks * kKBytes, &tmK, smem_u32(k_full + ks), 0, j * 64, bh);
+          ++tK;
+          if (++ks == kKStages) {
+            ks = 0;
+            kph ^= 1;
+          }
+          if (!have_next) nsteps = tK;
+          have = have_next;
+          j = jn;
+          fl = fln;
+          progress = true;
+        }
+        // V: the next step whose K has been issued, once its slot is free
+        if (tV < tK && (tV < kVStages || mbar_test_wait(smem_u32(v_empty + vs), vph ^ 1))) {
+          const int jv = meta[tV % kKStages].j;  // K slot of step tV: not reused before V(tV)
+          mbar_expect_tx(smem_u32(v_full + vs), kVBytes);
+          tma_load_3d(sV + vs * kVBytes, &tmV, smem_u32(v_full + vs), 0, jv * 64, bh);
+          tma_load_3d(sV + vs * kVBytes + 8192, &tmV, smem_u32(v_full + vs), 64, jv * 64, bh);
+          ++tV;
+          if (++vs == kVStages) {
+            vs = 0;
+            vph ^= 1;
+          }
+          progress = true;
+        }
+        if (nsteps >= 0 && tV == nsteps) break;
+        if (progress) {
+          t_idle = 0;
+          continue;
+        }
+        // nothing to issue: sleep on the V slot we need next (the usual blocker)
+        if (tV < tK && tV >= kVStages) mbar_try_wait_suspend(smem_u32(v_empty + vs), vph ^ 1, 2000u);
+        else if (tK >= kKStages) mbar_try_wait_suspend(smem_u32(k_empty + ks), kph ^ 1, 2000u);
+        if (abort_flag) {
           aborted = true;
           break;
         }
-        meta[s].j = j;
-        meta[s].flags = fl | (have_next ? 0 : 4);
-        meta[s].sk = __ldg(p.k_scale + static_cast<size_t>(bh) * nB + j);
-        const uint32_t dst = sStage + s * kStageBytes;
-        mbar_expect_tx(smem_u32(kv_full + s), kStageBytes);
-        tma_load_3d(dst, &tmK, smem_u32(kv_full + s), 0, j * 64, bh);
-        tma_load_3d(dst + 8192, &tmV, smem_u32(kv_full + s), 0, j * 64, bh);
-        tma_load_3d(dst + 16384, &tmV, smem_u32(kv_full + s), 64, j * 64, bh);
-        ++t;
-        have = have_next;
-        j = jn;
-        fl = fln;
+        const unsigned long long now = globaltimer();
+        if (t_idle == 0) {
+          t_idle = now;
+        } else if (now - t_idle > kWaitLimitNs) {
+          abort_flag = 1;
+          atomicOr(p.status, kStatusTimeout);
+          aborted = true;
+          break;
+        }
       }
       if (aborted || abort_flag) {  // let the copies in flight land before exit
         mbar_drain(smem_u32(q_full), 0, p.status);
-        for (int u = max(0, t - kStages); u < t; ++u)
-          mbar_drain(smem_u32(kv_full + (u % kStages)), (u / kStages) & 1, p.status);
+        for (int u = max(0, tK - kKStages); u < tK; ++u)
+          mbar_drain(smem_u32(k_full + (u % kKStages)), (u / kKStages) & 1, p.status);
+        for (int u = max(0, tV - kVStages); u < tV; ++u)
+          mbar_drain(smem_u32(v_full + (u % kVStages)), (u / kVStages) & 1, p.status);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // Issue order QK(0), QK(1), PV(0), QK(2), PV(1), ...: tcgen05.mma ops from one thread
     // execute in issue order, so QK(t) overwriting S_(t%2) (which holds P(t-2)) runs after
-    // PV(t-2) has read it.
+    // PV(t-2) has read it. PV waits only for the halves that are critical for its step and
+    // masks the D lanes of the other half.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = make_idesc(2, 1, 0, 0, 128, 64);
       constexpr uint32_t idesc_pv = make_idesc(1, 1, 0, 1, 128, 128);
+      const uint64_t dq = make_sdesc(sQ, 16, 1024);
+      const uint64_t dk0 = make_sdesc(sK, 16, 1024);
+      const uint64_t dv0 = make_sdesc(sV, 8192, 1024);
+      constexpr uint64_t kKDesc = kKBytes >> 4;  // start-address field units (16 B)
+      constexpr uint64_t kVDesc = kVBytes >> 4;
       bool ok = mbar_wait(smem_u32(q_full), 0, &abort_flag, p.status);
-      auto issue_pv = [&](int u) -> bool {
-        const int s = u % kStages, b = u & 1;
-        if (!mbar_wait(smem_u32(p_full + b), (u >> 1) & 1, &abort_flag, p.status)) return false;
+      int pcnt[2][2] = {{0, 0}, {0, 0}};  // completed p_full phases per (half, buffer)
+      int prev_flags = 0;
+      int vs = 0, vph = 0;
+      auto issue_pv = [&](int u, int fl) -> bool {
+        const int b = u & 1;
+        if (!mbar_wait(smem_u32(v_full + vs), vph, &abort_flag, p.status)) return false;
+        for (int h = 0; h < 2; ++h) {
+          if (fl & (1 << h)) {
+            if (!mbar_wait(smem_u32(p_full + 2 * h + b), pcnt[h][b] & 1, &abort_flag, p.status))
+              return false;
+            ++pcnt[h][b];
+          }
+        }
         tc_fence_after();
-        const uint32_t v = sStage + s * kStageBytes + 8192;
+        const uint32_t m01 = (fl & 1) ? 0u : 0xffffffffu;  // disable lanes 0-63 if half 0 is out
+        const uint32_t m23 = (fl & 2) ? 0u : 0xffffffffu;
+        const uint64_t dv = dv0 + kVDesc * vs;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ts(taddr + kColO, taddr + 64 * b + 8 * kk, make_sdesc(v + kk * 2048, 8192, 1024),
-                      idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(smem_u32(kv_empty + s));
+          mma_bf16_ts_masked(taddr + kColO, taddr + 64 * b + 8 * kk, dv + 128 * kk, idesc_pv, 1u,
+                             m01, m01, m23, m23);
+        mma_commit(smem_u32(v_empty + vs));
         mma_commit(smem_u32(pv_done + b));
+        if (++vs == kVStages) {
+          vs = 0;
+          vph ^= 1;
+        }
         return true;
       };
-      int t = 0;
+      int t = 0, s = 0, ph = 0;
       bool last = false;
       while (ok && !last) {
-        const int s = t % kStages, b = t & 1;
-        if (!mbar_wait(smem_u32(kv_full + s), (t / kStages) & 1, &abort_flag, p.status)) {
+        const int b = t & 1;
+        if (!mbar_wait(smem_u32(k_full + s), ph, &abort_flag, p.status)) {
           ok = false;
           break;
         }
-        last = (meta[s].flags & 4) != 0;
+        const int fl = meta[s].flags;
+        last = (fl & 4) != 0;
         tc_fence_after();
-        const uint32_t kt = sStage + s * kStageBytes;
+        const uint64_t dk = dk0 + kKDesc * s;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_i8(taddr + 64 * b, make_sdesc(sQ + kk * 32, 16, 1024), make_sdesc(kt + kk * 32, 16, 1024),
-                 idesc_qk, kk > 0 ? 1u : 0u);
-        mma_commit(smem_u32(s_full + b));
-        if (t >= 1 && !issue_pv(t - 1)) {
+          mma_i8(taddr + 64 * b, dq + 2 * kk, dk + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
+        mma_commit(smem_u32(k_empty + s));
+        mma_commit(smem_u32(s_full + (t & 7)));
+        if (t >= 1 && !issue_pv(t - 1, prev_flags)) {
           ok = false;
           break;
         }
+        prev_flags = fl;
         ++t;
+        if (++s == kKStages) {
+          s = 0;
+          ph ^= 1;
+        }
       }
-      if (ok && t >= 1) ok = issue_pv(t - 1);
+      if (ok && t >= 1) ok = issue_pv(t - 1, prev_flags);
       mma_commit(smem_u32(o_full));
       mbar_drain(smem_u32(o_full), 0, p.status);
     }
@@ -403,7 +516,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     // Warp w owns the 16 TMEM lanes LB = 32*(w%4) + 16*((w-2)/4) .. LB+15 (query rows of the
     // 128-row tile); in the 16-lane load shape thread t holds rows LB + t/4 and LB + t/4 + 8,
     // 16 keys each, and the four threads of a quad (t/4) share rows. Rows 0-63 are block i0,
-    // 64-127 block i0+1, so membership is warp-uniform.
+    // 64-127 block i0+1, so membership is warp-uniform. A warp whose half is not critical
+    // for a step skips it (the P.V MMA masks its rows).
     const int wq = warp & 3;
     const int sub = (warp - 2) >> 2;
     const uint32_t lb = 32 * wq + 16 * sub;
@@ -413,25 +527,38 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const int i = i0 + half;
     const float sq = (i < nB) ? p.q_scale[static_cast<size_t>(bh) * nB + i] : 0.f;
     const uint32_t lane_off = lb << 16;
+    {  // O starts at zero for these rows; every P.V then accumulates
+      uint32_t z[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) z[c] = 0u;
+      tmem_st_16x256b_x8(taddr + lane_off + kColO, z);
+      tmem_st_16x256b_x8(taddr + lane_off + kColO + 64, z);
+      tmem_wait_st();
+    }
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     bool ok = true;
     bool last = false;
-    int t = 0;
+    int t = 0, s = 0, ph = 0;
     while (!last) {
-      const int b = t & 1, s = t % kStages;
-      ok = mbar_wait(smem_u32(s_full + b), (t >> 1) & 1, &abort_flag, p.status);
-      ok = ok && mbar_wait(smem_u32(kv_full + s), (t / kStages) & 1, &abort_flag, p.status);
+      const int b = t & 1;
+      ok = mbar_wait(smem_u32(k_full + s), ph, &abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
-      tc_fence_after();
       const int j = meta[s].j, fl = meta[s].flags;
       const float skj = meta[s].sk;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(k_empty + s));
       last = (fl & 4) != 0;
       const bool member = (fl >> half) & 1;  // warp-uniform
-      uint32_t pk[16];
       if (member) {
+        ok = mbar_wait(smem_u32(s_full + (t & 7)), (t >> 3) & 1, &abort_flag, p.status);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         uint32_t sv[32];
         tmem_ld_16x256b_x8(taddr + lane_off + 64 * b, sv);
         const bool ragged = (j == nB - 1) && (p.N - j * 64 < 64);  // CTA-uniform
@@ -439,26 +566,24 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         float A[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) A[c] = __int_as_float(static_cast<int>(sv[c]) + kMagicBits);
-        float mA0 = 0.f, mA1 = 0.f;  // 0 is below every real value (all >= 1.5*2^23 - 2^22)
-        if (!ragged) {
-          mA0 = fmax3(A[0], A[1], A[4]);
-          mA1 = fmax3(A[2], A[3], A[6]);
-          mA0 = fmax3(mA0, A[5], A[8]);
-          mA1 = fmax3(mA1, A[7], A[10]);
+        const float sc = __fmul_rn(__fmul_rn(sq, skj), kLog2e);
+        uint32_t pk[16];
+        float ps0, ps1;
+        if (ragged)
+          softmax_tile<true>(A, sc, -m0, -m1, q, nvalid, pk, ps0, ps1);
+        else
+          softmax_tile<false>(A, sc, -m0, -m1, q, 64, pk, ps0, ps1);
+        // rare path: raise m where a partial sum left [0, 2^24] (quad-consistent decision)
+        bool need0 = !(ps0 <= kPsumLimit), need1 = !(ps1 <= kPsumLimit);
+        need0 = quad_any(need0);
+        need1 = quad_any(need1);
+        float alpha0 = 1.f, alpha1 = 1.f;
+        if (__any_sync(0xffffffffu, need0 || need1)) {
+          // S_b still holds the scores (P overwrites it only below): reload them.
+          tmem_ld_16x256b_x8(taddr + lane_off + 64 * b, sv);
 #pragma unroll
-          for (int k = 2; k < 8; ++k) {
-            if (k == 2) {
-              mA0 = fmax3(mA0, A[9], A[12]);
-              mA1 = fmax3(mA1, A[11], A[14]);
-            } else if (k < 7) {
-              mA0 = fmax3(mA0, A[4 * k + 1], A[4 * k + 4]);
-              mA1 = fmax3(mA1, A[4 * k + 3], A[4 * k + 6]);
-            } else {
-              mA0 = fmaxf(mA0, A[29]);
-              mA1 = fmaxf(mA1, A[31]);
-            }
-          }
-        } else {
+          for (int c = 0; c < 32; ++c) A[c] = __int_as_float(static_cast<int>(sv[c]) + kMagicBits);
+          float mA0 = 0.f, mA1 = 0.f;  // 0 is below every real value (all >= 1.5*2^23 - 2^22)
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const int c = 8 * k + 2 * q;
@@ -471,27 +596,28 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
               mA1 = fmaxf(mA1, A[4 * k + 3]);
             }
           }
+          mA0 = quad_max(mA0);
+          mA1 = quad_max(mA1);
+          if (need0) {
+            const float mt = __fmul_rn(__fsub_rn(mA0, kMagic), sc);
+            if (m0 != -INFINITY) alpha0 = ex2_approx(m0 - mt);
+            m0 = mt;
+          }
+          if (need1) {
+            const float mt = __fmul_rn(__fsub_rn(mA1, kMagic), sc);
+            if (m1 != -INFINITY) alpha1 = ex2_approx(m1 - mt);
+            m1 = mt;
+          }
+          if (ragged)
+            softmax_tile<true>(A, sc, -m0, -m1, q, nvalid, pk, ps0, ps1);
+          else
+            softmax_tile<false>(A, sc, -m0, -m1, q, 64, pk, ps0, ps1);
         }
-        mA0 = quad_max(mA0);
-        mA1 = quad_max(mA1);
-        const float sc = __fmul_rn(__fmul_rn(sq, skj), kLog2e);
-        const float mt0 = __fmul_rn(__fsub_rn(mA0, kMagic), sc);
-        const float mt1 = __fmul_rn(__fsub_rn(mA1, kMagic), sc);
-        const bool raise0 = mt0 > m0 + kRescaleThreshold, raise1 = mt1 > m1 + kRescaleThreshold;
-        const bool resc0 = raise0 && (m0 != -INFINITY), resc1 = raise1 && (m1 != -INFINITY);
-        const float alpha0 = resc0 ? ex2_approx(m0 - mt0) : 1.f;
-        const float alpha1 = resc1 ? ex2_approx(m1 - mt1) : 1.f;
-        if (raise0) m0 = mt0;
-        if (raise1) m1 = mt1;
-        float ps0, ps1;
-        if (ragged)
-          softmax_tile<true>(A, sc, -m0, -m1, q, nvalid, pk, ps0, ps1);
-        else
-          softmax_tile<false>(A, sc, -m0, -m1, q, 64, pk, ps0, ps1);
         l0 = fmaf(l0, alpha0, ps0);
         l1 = fmaf(l1, alpha1, ps1);
-        if (__any_sync(0xffffffffu, resc0 || resc1)) {
-          // O holds P.V of earlier tiles: wait for the last issued P.V, then rescale rows.
+        tmem_st_16x128b_x8(taddr + lane_off + 64 * b, pk);  // P first: its registers die here
+        if (__any_sync(0xffffffffu, alpha0 != 1.f || alpha1 != 1.f)) {
+          // O holds P.V of earlier steps: wait for the last issued P.V, then rescale rows.
           if (t >= 1)
             ok = mbar_wait(smem_u32(pv_done + ((t - 1) & 1)), ((t - 1) >> 1) & 1, &abort_flag,
                            p.status);
@@ -514,17 +640,16 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             }
             tmem_st_16x256b_x8(oa, o);
           }
-          tmem_wait_st();
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 16; ++c) pk[c] = 0u;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_u32(p_full + 2 * half + b));
       }
-      tmem_st_16x128b_x8(taddr + lane_off + 64 * b, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(smem_u32(p_full + b));
       ++t;
+      if (++s == kKStages) {
+        s = 0;
+        ph ^= 1;
+      }
     }
 
     // ------------------------------------------------------------ epilogue
