@@ -40,6 +40,31 @@ def dense_equiv_ops(wl) -> float:
     return 4.0 * wl.B * wl.H * float(wl.N) ** 2 * wl.d
 
 
+def profiled_traffic(workload: str):
+    """DRAM bytes per attn_kernel launch from the committed ncu summary, or None.
+
+    The summary records the sha256 prefix of the kernel source it was taken on; once the
+    source has changed the counters no longer describe the kernel and None is returned.
+    """
+    import hashlib
+    summary = os.path.join(ROOT, "profiles", f"attn_kernel_{workload}.md")
+    src = os.path.join(ROOT, "quantized_block_sparse_b200", "csrc", "attention.cu")
+    if not (os.path.exists(summary) and os.path.exists(src)):
+        return None
+    fields = {}
+    with open(summary) as f:
+        for line in f:
+            if ":" in line and not line.startswith(("|", "#", " ")):
+                key, _, val = line.partition(":")
+                fields[key.strip()] = val.strip()
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    prefix = fields.get("source_sha256_prefix")
+    if not prefix or not sha.startswith(prefix) or "dram_bytes_per_launch" not in fields:
+        return None
+    return int(fields["dram_bytes_per_launch"])
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -50,13 +75,14 @@ def load_peaks():
 
 
 # ------------------------------------------------------------------ CPU oracle timing
-def oracle_sample(q, k, v, wl, n_small=4, n_large=12):
-    """Time the CPU oracle on one head and extrapolate to the whole call.
+def oracle_sample(q, k, v, wl, n_small=None, n_large=None):
+    """Time the CPU oracle on one head and scale to the whole call.
 
-    Per head the oracle does prepare + select (fixed) and forward over nB query blocks.
-    forward(head, S blocks) is timed for two block-set sizes; a linear fit a + b*|S|
-    splits its per-head fixed part (linear states, H = M h) from the per-block part.
-    Estimate of one call: B*H * (t_prep_sel + a + b * nB).
+    Default (the cpu_baseline leg): one whole head, prepare + select + forward over all
+    nB query blocks; call time = B*H * that (heads are independent and equal in work).
+    With n_small/n_large (the per-step sample of --impl reference): forward runs on two
+    block-set sizes and a linear fit a + b*|S| splits the per-head fixed part (linear
+    states, H = M h) from the per-block part; call time = B*H * (prep_sel + a + b*nB).
     """
     import oracle as O
     from threadpoolctl import threadpool_info
@@ -69,25 +95,35 @@ def oracle_sample(q, k, v, wl, n_small=4, n_large=12):
     prep = O.prepare(qf, kf)
     sel = O.select(prep.q_bar, prep.k_bar, wl.rho, wl.nu)
     t_ps = time.perf_counter() - t0
-    rng = np.random.default_rng(0)
-    ts = []
-    for n in (n_small, n_large):
-        blocks = sorted(rng.choice(nB, size=min(n, nB), replace=False).tolist())
+    if n_small is None:
         t1 = time.perf_counter()
-        O.forward(prep, vf, sel, heads=[(0, 0)], qblocks=blocks)
-        ts.append((len(blocks), time.perf_counter() - t1))
-    (n1, t1), (n2, t2) = ts
-    b = max((t2 - t1) / max(n2 - n1, 1), 0.0)
-    a = max(t1 - b * n1, 0.0)
-    per_head = t_ps + a + b * nB
+        O.forward(prep, vf, sel, heads=[(0, 0)])
+        t_fwd = time.perf_counter() - t1
+        per_head = t_ps + t_fwd
+        wall = per_head
+        sample = (f"1 of {wl.B * wl.H} heads, whole: prepare+select+forward over all {nB} query "
+                  f"blocks ({wall:.1f} s of CPU work); call time = B*H * per-head time")
+    else:
+        rng = np.random.default_rng(0)
+        ts = []
+        for n in (n_small, n_large):
+            blocks = sorted(rng.choice(nB, size=min(n, nB), replace=False).tolist())
+            t1 = time.perf_counter()
+            O.forward(prep, vf, sel, heads=[(0, 0)], qblocks=blocks)
+            ts.append((len(blocks), time.perf_counter() - t1))
+        (n1, t1), (n2, t2) = ts
+        b = max((t2 - t1) / max(n2 - n1, 1), 0.0)
+        a = max(t1 - b * n1, 0.0)
+        per_head = t_ps + a + b * nB
+        wall = t_ps + t1 + t2
+        sample = (f"1 of {wl.B * wl.H} heads: prepare+select, forward on {n1} and {n2} of {nB} "
+                  f"query blocks; call time extrapolated as B*H*(prep_sel + a + b*nB); "
+                  f"{wall:.1f} s of CPU work")
     est_s = wl.B * wl.H * per_head
     cores = 0
     for info in threadpool_info():
         cores = max(cores, int(info.get("num_threads", 0)))
     cores = cores or os.cpu_count()
-    wall = t_ps + t1 + t2
-    sample = (f"1 of {wl.B * wl.H} heads: prepare+select, forward on {n1} and {n2} of {nB} query "
-              f"blocks; call time extrapolated as B*H*(prep_sel + a + b*nB); {wall:.1f} s of CPU work")
     return est_s, cores, sample
 
 
@@ -298,9 +334,11 @@ def run_ours(args, wl):
         "roofline": {"kernel": "attn_kernel", "bound": "tensor", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak,
-                     "traffic": None,
+                     "traffic": profiled_traffic(wl.name),
                      "note": (f"bf16-equivalent: INT8 QK^T ops / {INT8_TO_BF16_RATE:g} + BF16 PV flops over "
-                              f"{pairs} executed 64x64 block pairs; peak = {peak_src} cuBLAS bf16 burst")},
+                              f"{pairs} executed 64x64 block pairs; peak = {peak_src} cuBLAS bf16 burst; "
+                              f"traffic = DRAM bytes per launch from the committed ncu summary "
+                              f"(null once the kernel source differs from the profiled one)")},
         "e2e": {"value": dense_ops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(round(launches_per_step * args.steps)),
