@@ -11,7 +11,7 @@
 //   hgemm_kernel   H = M . h per head, M the 0/1 marginal mask [nB x nBp] and h viewed as
 //                  [nB x d*d]: a tcgen05 bf16 GEMM (fp32 accumulation in TMEM), 128x128
 //                  output tiles, TMA-fed 3-stage pipeline, bf16 output.
-//   zsum_kernel    Z_i = sum of z_j over the marginal list, fp32, ascending j.
+//   zsum_kernel    Z_i = sum of z_j over the marginal blocks (mask row), fp32, ascending j.
 //   linout_kernel  per pair of query blocks: phi(Q~) (recomputed from Q, bf16) times H_i
 //                  on tcgen05 (M = 128 rows = both blocks, one MMA chain per block),
 //                  divided by phi(Q~) . Z_i; bf16 O_l for the attention epilogue.
@@ -119,15 +119,64 @@ __global__ void __launch_bounds__(128) hgemm_kernel(const __grid_constant__ CUte
 }
 
 // ------------------------------------------------------------------ Z_i
-__global__ void __launch_bounds__(128) zsum_kernel(const float* __restrict__ z,
-                                                   const int32_t* __restrict__ marg,
-                                                   float* __restrict__ Z, int nB, int m) {
-  const int i = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
-  const int32_t* ml = marg + (static_cast<size_t>(bh) * nB + i) * m;
-  const float* zb = z + static_cast<size_t>(bh) * nB * kHeadDim + c;
-  float acc = 0.f;
-  for (int t = 0; t < m; ++t) acc += zb[static_cast<size_t>(ml[t]) * kHeadDim];
-  Z[(static_cast<size_t>(bh) * nB + i) * kHeadDim + c] = acc;
+// Z_i = sum over j of mask_ij * z_j, ascending j, one fp32 FMA per term (mask_ij is 0 or 1,
+// so each step adds z_j exactly once or leaves the sum unchanged). A CTA covers 16 query
+// blocks; z and the mask rows are staged in shared memory 128 key blocks at a time, so each
+// z row is read from L2 once per 16 query blocks instead of once per query block.
+constexpr int kZRows = 16;
+constexpr int kZChunk = 128;
+constexpr int kZSmem = (kZChunk * kHeadDim + kZRows * kZChunk) * 4;
+
+__global__ void __launch_bounds__(256) zsum_kernel(const float* __restrict__ z,
+                                                   const __nv_bfloat16* __restrict__ mask,
+                                                   float* __restrict__ Z, int nB, int nBp) {
+  extern __shared__ float zsm[];
+  float* zs = zsm;                          // [kZChunk][128]
+  float* ms = zsm + kZChunk * kHeadDim;     // [kZRows][kZChunk]
+  const int i0 = blockIdx.x * kZRows, bh = blockIdx.y, tid = threadIdx.x;
+  const int g = tid >> 7, c = tid & 127;
+  const int rows = min(kZRows, nB - i0);
+  const float* zh = z + static_cast<size_t>(bh) * nB * kHeadDim;
+  const __nv_bfloat16* mh = mask + (static_cast<size_t>(bh) * nB + i0) * nBp;
+  float acc[kZRows / 2];
+#pragma unroll
+  for (int r = 0; r < kZRows / 2; ++r) acc[r] = 0.f;
+
+  for (int j0 = 0; j0 < nB; j0 += kZChunk) {
+    const int jn = min(kZChunk, nB - j0), jn4 = (jn + 3) & ~3;
+    __syncthreads();
+    const float4* src = reinterpret_cast<const float4*>(zh + static_cast<size_t>(j0) * kHeadDim);
+    for (int x = tid; x < jn * (kHeadDim / 4); x += 256) cp_async16(smem_u32(zs + 4 * x), src + x);
+    cp_async_commit();
+    for (int x = jn * (kHeadDim / 4) + tid; x < jn4 * (kHeadDim / 4); x += 256)
+      reinterpret_cast<float4*>(zs)[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int t = 0; t < kZRows * kZChunk / 256; ++t) {
+      const int x = tid + 256 * t;
+      const int r = x / kZChunk, jj = x % kZChunk;
+      ms[x] = (r < rows && jj < jn) ? __bfloat162float(mh[static_cast<size_t>(r) * nBp + j0 + jj]) : 0.f;
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    const float* mrow = ms + g * (kZRows / 2) * kZChunk;
+    for (int jj = 0; jj < jn4; jj += 4) {
+      const float z0 = zs[(jj + 0) * kHeadDim + c], z1 = zs[(jj + 1) * kHeadDim + c];
+      const float z2 = zs[(jj + 2) * kHeadDim + c], z3 = zs[(jj + 3) * kHeadDim + c];
+#pragma unroll
+      for (int r = 0; r < kZRows / 2; ++r) {
+        const float4 mv = *reinterpret_cast<const float4*>(mrow + r * kZChunk + jj);
+        acc[r] = fmaf(mv.x, z0, acc[r]);
+        acc[r] = fmaf(mv.y, z1, acc[r]);
+        acc[r] = fmaf(mv.z, z2, acc[r]);
+        acc[r] = fmaf(mv.w, z3, acc[r]);
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < kZRows / 2; ++r) {
+    const int row = g * (kZRows / 2) + r;
+    if (row < rows) Z[(static_cast<size_t>(bh) * nB + i0 + row) * kHeadDim + c] = acc[r];
+  }
 }
 
 // ------------------------------------------------------------------ O_l
@@ -278,6 +327,8 @@ cudaError_t launch_linear(const Dims& g, const void* q, float sm_scale, const vo
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(linout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem);
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(zsum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kZSmem);
+  if (e != cudaSuccess) return e;
 
   {
     TraceScope ts_("hgemm_kernel", st);
@@ -286,7 +337,8 @@ cudaError_t launch_linear(const Dims& g, const void* q, float sm_scale, const vo
   }
   {
     TraceScope ts_("zsum_kernel", st);
-    zsum_kernel<<<dim3(g.nB, g.BH), 128, 0, st>>>(z, marg, Zbuf, g.nB, m);
+    zsum_kernel<<<dim3((g.nB + kZRows - 1) / kZRows, g.BH), 256, kZSmem, st>>>(
+      z, static_cast<const __nv_bfloat16*>(mask), Zbuf, g.nB, g.nBp);
   }
   {
     TraceScope ts_("linout_kernel", st);

@@ -76,18 +76,29 @@ struct PrepParams {
 };
 
 constexpr int kPrepThreads = 256;
-constexpr int kPrepSmem = 16384 + 16384 + 64 * 128 * 4 + 1024 + 256;
+// V tile (MN-major SW128, TMA), phi(K~)^T tile (K-major SW128), raw Q and K blocks (bulk
+// copies), reduction scratch and barriers.
+constexpr int kPrepSmem = 4 * 16384 + 256 + 1024;
 
-__device__ __forceinline__ float block_max(float v, float* red) {
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+// Block max of two values at once (Q and K amax); every thread gets both results.
+__device__ __forceinline__ float2 block_max2(float a, float b, float* red) {
+  for (int o = 16; o > 0; o >>= 1) {
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    red[warp] = a;
+    red[8 + warp] = b;
+  }
   __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  float m = red[0];
+  float ma = red[0], mb = red[8];
 #pragma unroll
-  for (int w = 1; w < kPrepThreads / 32; ++w) m = fmaxf(m, red[w]);
-  return m;
+  for (int w = 1; w < kPrepThreads / 32; ++w) {
+    ma = fmaxf(ma, red[w]);
+    mb = fmaxf(mb, red[8 + w]);
+  }
+  return make_float2(ma, mb);
 }
 
 __device__ __forceinline__ int quant_code(float x, float s) {
@@ -96,24 +107,7 @@ __device__ __forceinline__ int quant_code(float x, float s) {
   return max(-127, min(127, c));
 }
 
-// Quantize this thread's 4 rows x 8 channels and store 8 codes per row.
-__device__ __forceinline__ void store_codes(const float (&x)[4][8], float s, int8_t* dst_rows,
-                                            int rg, int chunk) {
-#pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
-    const int r = rg + 16 * kk;
-    uint32_t lo = 0, hi = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      lo |= (static_cast<uint32_t>(quant_code(x[kk][e], s)) & 0xffu) << (8 * e);
-      hi |= (static_cast<uint32_t>(quant_code(x[kk][e + 4], s)) & 0xffu) << (8 * e);
-    }
-    *reinterpret_cast<uint2*>(dst_rows + r * kHeadDim + 8 * chunk) = make_uint2(lo, hi);
-  }
-}
-
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4*>(p);
+__device__ __forceinline__ void unpack8(const uint4 u, float (&f)[8]) {
   const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
@@ -125,16 +119,21 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
 
 __device__ __forceinline__ float phi_f32(float x) { return x > 0.f ? __fadd_rn(x, 1.f) : expf(x); }
 
-__global__ void __launch_bounds__(kPrepThreads) prep_block_kernel(PrepParams p) {
+// One CTA per (head, 64-token block). All three input blocks are requested at once (two
+// bulk copies for the raw Q and K rows, two TMA boxes for V straight into the MN-major
+// 128-byte-swizzled operand tile), so a CTA keeps 48 KB in flight and three CTAs share an SM.
+__global__ void __launch_bounds__(kPrepThreads, 3) prep_block_kernel(const __grid_constant__ CUtensorMap tmV,
+                                                                   PrepParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  unsigned char* sA = smem;          // phi(K~)^T: 128 rows (c) x 64 tokens, K-major, SW128
-  unsigned char* sB = smem + 16384;  // V: 2 groups x 64 tokens x 64 e, MN-major, SW128
-  float* xs = reinterpret_cast<float*>(smem + 32768);  // [64][128] fp32 staging
-  float* red = xs + 64 * 128;                          // [8]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(red + 8);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+  unsigned char* sB = smem;          // V: 2 groups x 64 tokens x 64 e, MN-major, SW128
+  unsigned char* sA = smem + 16384;  // phi(K~)^T: 128 rows (c) x 64 tokens, K-major, SW128
+  const __nv_bfloat16* sQ = reinterpret_cast<const __nv_bfloat16*>(smem + 32768);  // [64][128]
+  const __nv_bfloat16* sK = reinterpret_cast<const __nv_bfloat16*>(smem + 49152);  // [64][128]
+  float* red = reinterpret_cast<float*>(smem + 65536);                              // [16]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(red + 16);  // [0] inputs landed, [1] MMA done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 2);
   __shared__ int abort_flag;
 
   const int j = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -148,81 +147,76 @@ __global__ void __launch_bounds__(kPrepThreads) prep_block_kernel(PrepParams p) 
   if (tid == 0) {
     abort_flag = 0;
     mbar_init(smem_u32(bar), 1);
+    mbar_init(smem_u32(bar + 1), 1);
     fence_mbar_init();
+    const uint32_t rows_bytes = static_cast<uint32_t>(n) * kHeadDim * 2;
+    mbar_expect_tx(smem_u32(bar), 2 * rows_bytes + 16384);
+    bulk_load(smem_u32(sQ), p.q + row0 * kHeadDim, rows_bytes, smem_u32(bar));
+    bulk_load(smem_u32(sK), p.k + row0 * kHeadDim, rows_bytes, smem_u32(bar));
+    tma_load_3d(smem_u32(sB), &tmV, smem_u32(bar), 0, j * kBlock, bh);
+    tma_load_3d(smem_u32(sB) + 8192, &tmV, smem_u32(bar), 64, j * kBlock, bh);
   }
-
-  // ---------------- Q: scale, quantize, block mean
-  float x[4][8];
-  float lmax = 0.f;
-#pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
-    const int r = rg + 16 * kk;
-    if (r < n) {
-      load8(p.q + (row0 + r) * kHeadDim + 8 * chunk, x[kk]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[kk][e] = __fmul_rn(x[kk][e], p.c_s);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[kk][e] = 0.f;
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      xs[r * kHeadDim + 8 * chunk + e] = x[kk][e];
-      lmax = fmaxf(lmax, fabsf(x[kk][e]));
-    }
-  }
-  float s = __fdiv_rn(block_max(lmax, red), 127.f);
-  store_codes(x, s, p.q8 + prow0 * kHeadDim, rg, chunk);
-  if (tid == 0) p.q_scale[blk] = s;
-  if (tid < kHeadDim) {
-    float acc = 0.f;
-    for (int r = 0; r < n; ++r) acc = __fadd_rn(acc, xs[r * kHeadDim + tid]);
-    p.q_bar[blk * kHeadDim + tid] = __fdiv_rn(acc, static_cast<float>(n));
-  }
-  __syncthreads();
-
-  // ---------------- K: smooth, quantize, block mean, phi(K~) for the linear state
-  lmax = 0.f;
   float mu8[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) mu8[e] = p.mu[bh * kHeadDim + 8 * chunk + e];
+  const float mu_c = p.mu[bh * kHeadDim + (tid & 127)];
+  __syncthreads();
+  if (!mbar_wait(smem_u32(bar), 0, &abort_flag, p.status)) mbar_wait_inflight(smem_u32(bar), 0, p.status);
+
+  // ---------------- Q~ = Q*c_s and K~ = K-mu: scales and INT8 codes (4 rows x 8 channels).
+  // The fp32 values are recomputed from the shared-memory rows for the codes instead of
+  // being held across the block reduction (the same two fp32 operations give the same bits).
+  float lq = 0.f, lk = 0.f;
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk) {
     const int r = rg + 16 * kk;
     if (r < n) {
-      load8(p.k + (row0 + r) * kHeadDim + 8 * chunk, x[kk]);
+      float fq[8], fk[8];
+      unpack8(*reinterpret_cast<const uint4*>(sQ + r * kHeadDim + 8 * chunk), fq);
+      unpack8(*reinterpret_cast<const uint4*>(sK + r * kHeadDim + 8 * chunk), fk);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) x[kk][e] = __fsub_rn(x[kk][e], mu8[e]);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[kk][e] = 0.f;
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      xs[r * kHeadDim + 8 * chunk + e] = x[kk][e];
-      lmax = fmaxf(lmax, fabsf(x[kk][e]));
+      for (int e = 0; e < 8; ++e) {
+        lq = fmaxf(lq, fabsf(__fmul_rn(fq[e], p.c_s)));
+        lk = fmaxf(lk, fabsf(__fsub_rn(fk[e], mu8[e])));
+      }
     }
   }
-  s = __fdiv_rn(block_max(lmax, red), 127.f);
-  store_codes(x, s, p.k8 + prow0 * kHeadDim, rg, chunk);
-  if (tid == 0) p.k_scale[blk] = s;
-
-  // V rows -> MN-major SW128 tile (zeros for padded tokens)
+  const float2 amax = block_max2(lq, lk, red);
+  const float sq = __fdiv_rn(amax.x, 127.f), sk = __fdiv_rn(amax.y, 127.f);
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk) {
     const int r = rg + 16 * kk;
-    uint4 u = make_uint4(0, 0, 0, 0);
-    if (r < n) u = *reinterpret_cast<const uint4*>(p.v + (row0 + r) * kHeadDim + 8 * chunk);
-    st_shared_v4(smem_u32(sB) + (chunk >> 3) * 8192 + sw128_offset(r, chunk & 7), u.x, u.y, u.z,
-                 u.w);
+    uint32_t cq[2] = {0u, 0u}, ck[2] = {0u, 0u};
+    if (r < n) {
+      float fq[8], fk[8];
+      unpack8(*reinterpret_cast<const uint4*>(sQ + r * kHeadDim + 8 * chunk), fq);
+      unpack8(*reinterpret_cast<const uint4*>(sK + r * kHeadDim + 8 * chunk), fk);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        cq[e >> 2] |= (static_cast<uint32_t>(quant_code(__fmul_rn(fq[e], p.c_s), sq)) & 0xffu) << (8 * (e & 3));
+        ck[e >> 2] |= (static_cast<uint32_t>(quant_code(__fsub_rn(fk[e], mu8[e]), sk)) & 0xffu) << (8 * (e & 3));
+      }
+    }
+    *reinterpret_cast<uint2*>(p.q8 + (prow0 + r) * kHeadDim + 8 * chunk) = make_uint2(cq[0], cq[1]);
+    *reinterpret_cast<uint2*>(p.k8 + (prow0 + r) * kHeadDim + 8 * chunk) = make_uint2(ck[0], ck[1]);
+  }
+  if (tid == 0) {
+    p.q_scale[blk] = sq;
+    p.k_scale[blk] = sk;
   }
 
+  // ---------------- block means (warps 0-3) and phi(K~)^T, z (warps 4-7), channel c
+  const int c = tid & 127;
   float zacc = 0.f;
-  if (tid < kHeadDim) {
-    const int c = tid;
-    float acc = 0.f;
-    for (int r = 0; r < n; ++r) acc = __fadd_rn(acc, xs[r * kHeadDim + c]);
-    p.k_bar[blk * kHeadDim + c] = __fdiv_rn(acc, static_cast<float>(n));
+  if (tid < 128) {
+    float aq = 0.f, ak = 0.f;
+    for (int r = 0; r < n; ++r) {
+      aq = __fadd_rn(aq, __fmul_rn(__bfloat162float(sQ[r * kHeadDim + c]), p.c_s));
+      ak = __fadd_rn(ak, __fsub_rn(__bfloat162float(sK[r * kHeadDim + c]), mu_c));
+    }
+    p.q_bar[blk * kHeadDim + c] = __fdiv_rn(aq, static_cast<float>(n));
+    p.k_bar[blk * kHeadDim + c] = __fdiv_rn(ak, static_cast<float>(n));
+  } else {
     // row c of phi(K~)^T: 64 tokens, bf16, padded tokens 0
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -230,8 +224,9 @@ __global__ void __launch_bounds__(kPrepThreads) prep_block_kernel(PrepParams p) 
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int r0 = 8 * q + 2 * e;
-        const float f0 = r0 < n ? phi_f32(xs[r0 * kHeadDim + c]) : 0.f;
-        const float f1 = r0 + 1 < n ? phi_f32(xs[(r0 + 1) * kHeadDim + c]) : 0.f;
+        const float f0 = r0 < n ? phi_f32(__fsub_rn(__bfloat162float(sK[r0 * kHeadDim + c]), mu_c)) : 0.f;
+        const float f1 =
+            r0 + 1 < n ? phi_f32(__fsub_rn(__bfloat162float(sK[(r0 + 1) * kHeadDim + c]), mu_c)) : 0.f;
         zacc += f0 + f1;
         w[e] = pack_bf16x2(f0, f1);
       }
@@ -252,33 +247,26 @@ __global__ void __launch_bounds__(kPrepThreads) prep_block_kernel(PrepParams p) 
       const uint64_t b = make_sdesc(smem_u32(sB) + kk * 2048, 8192, 1024);
       mma_bf16(taddr, a, b, idesc, kk > 0);
     }
-    mma_commit(smem_u32(bar));
+    mma_commit(smem_u32(bar + 1));
   }
-  const bool ok = mbar_wait(smem_u32(bar), 0, &abort_flag, p.status);
+  if (!mbar_wait(smem_u32(bar + 1), 0, &abort_flag, p.status)) mbar_wait_inflight(smem_u32(bar + 1), 0, p.status);
   tc_fence_after();
 
   // h_j[c][e]: TMEM lane c, column e. Warps w and w+4 split the 128 columns.
-  if (ok) {
-    const int c = 32 * (warp & 3) + lane;
+  if (!abort_flag) {
+    const int cl = 32 * (warp & 3) + lane;
     const int col0 = 64 * (warp >> 2);
     uint32_t rr[64];
     tmem_ld64_sync(taddr + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + col0, rr);
-    uint4* dst = reinterpret_cast<uint4*>(p.h + (blk * kHeadDim + c) * kHeadDim + col0);
+    uint4* dst = reinterpret_cast<uint4*>(p.h + (blk * kHeadDim + cl) * kHeadDim + col0);
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
+    for (int q = 0; q < 8; ++q)
       dst[q] = make_uint4(pack_bf16x2(__uint_as_float(rr[8 * q]), __uint_as_float(rr[8 * q + 1])),
                           pack_bf16x2(__uint_as_float(rr[8 * q + 2]), __uint_as_float(rr[8 * q + 3])),
                           pack_bf16x2(__uint_as_float(rr[8 * q + 4]), __uint_as_float(rr[8 * q + 5])),
                           pack_bf16x2(__uint_as_float(rr[8 * q + 6]), __uint_as_float(rr[8 * q + 7])));
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      dst[4 + q] =
-          make_uint4(pack_bf16x2(__uint_as_float(rr[32 + 8 * q]), __uint_as_float(rr[32 + 8 * q + 1])),
-                     pack_bf16x2(__uint_as_float(rr[32 + 8 * q + 2]), __uint_as_float(rr[32 + 8 * q + 3])),
-                     pack_bf16x2(__uint_as_float(rr[32 + 8 * q + 4]), __uint_as_float(rr[32 + 8 * q + 5])),
-                     pack_bf16x2(__uint_as_float(rr[32 + 8 * q + 6]), __uint_as_float(rr[32 + 8 * q + 7])));
   }
-  if (tid < kHeadDim) p.z[blk * kHeadDim + tid] = zacc;
+  if (tid >= 128) p.z[blk * kHeadDim + c] = zacc;
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(taddr, 128);
@@ -302,6 +290,9 @@ cudaError_t launch_prepare(const Dims& g, const void* q, const void* k, const vo
     TraceScope ts_("kmean_kernel", st);
     kmean_kernel<<<dim3(g.BH, kHeadDim / 16), 256, 0, st>>>(part, k_mean, g.N, g.nB);
   }
+  CUtensorMap tmV;
+  if (!make_tmap_3d(&tmV, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim, g.N, g.BH, 64, 64))
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(prep_block_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem);
   if (e != cudaSuccess) return e;
@@ -325,7 +316,7 @@ cudaError_t launch_prepare(const Dims& g, const void* q, const void* k, const vo
   p.Npad = g.Npad;
   {
     TraceScope ts_("prep_block_kernel", st);
-    prep_block_kernel<<<dim3(g.nB, g.BH), kPrepThreads, kPrepSmem, st>>>(p);
+    prep_block_kernel<<<dim3(g.nB, g.BH), kPrepThreads, kPrepSmem, st>>>(tmV, p);
   }
   return cudaGetLastError();
 }

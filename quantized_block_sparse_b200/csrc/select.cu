@@ -5,16 +5,21 @@
 // covers the middle and the rest is skipped; section "Hands-On Tutorial": --sla_topk sets
 // the kept fraction (0.1 -> 90% sparsity).
 //
-// One CTA handles R query-block rows of one head:
+// One CTA handles R = 2*RT query-block rows of one head (two row groups of 128 threads):
 //   1. l_ij = fp32 dot of the block means in a fixed order (acc = 0; for c: acc =
-//      fl32(acc + fl32(qbar[c]*kbar[c]))) - no FMA, so any implementation following the
-//      order gets the same bits;
-//   2. each row's (l_ij, j) pairs are encoded as 64-bit keys that order by logit
-//      descending, then block index ascending, and sorted by a bitonic network in shared
-//      memory;
-//   3. sorted positions [0,k_c) are critical, [nB-n_neg, nB) negligible, the rest
-//      marginal; a warp-ballot compaction writes both lists in ascending block order and
-//      the 0/1 bf16 marginal mask row.
+//      fl32(acc + fl32(qbar[c]*kbar[c]))) - separate multiply and add, no FMA, so any
+//      implementation following the order gets the same bits. Each thread keeps an
+//      RT x 4 tile of (row, key block) fp32 accumulators; the key means are staged
+//      channel-major in shared memory, 16 channels at a time, by a double-buffered
+//      cp.async pipeline; the row means are read as broadcasts.
+//   2. Each row's logits become order-preserving 32-bit keys. One warp per row finds the
+//      k_c-th largest key T_c and the n_neg-th smallest key T_n by a most-significant-bit
+//      first search over the key bits (a warp-wide count per bit, stopping as soon as the
+//      count is exactly k_c). Total order: logit descending, block index ascending.
+//   3. Critical: key > T_c, plus the lowest-index blocks with key == T_c up to k_c in
+//      all. Negligible: key < T_n, plus the highest-index blocks with key == T_n up to
+//      n_neg. The rest is marginal. A warp-ballot compaction writes both lists in
+//      ascending block order and the 0/1 bf16 marginal mask row.
 #include "sagesla_internal.h"
 #include "sm100_primitives.cuh"
 
@@ -22,8 +27,15 @@ namespace sgs {
 namespace {
 
 constexpr int kSelThreads = 256;
-constexpr int kSelRowsMax = 16;
-constexpr int kSelKeys = 8192;  // R * nBpow keys per CTA (64 KB)
+constexpr int kGroupThreads = 128;                    // threads per row group (two groups)
+constexpr int kJPerThread = 4;                        // key blocks per thread per pass
+constexpr int kJPass = kGroupThreads * kJPerThread;   // 512 key blocks per pass
+constexpr int kChunk = 16;                            // channels per pipeline stage
+constexpr int kKStride = kJPass + 4;                  // floats per staged channel row
+constexpr int kStages = kHeadDim / kChunk;            // 8 stages per pass
+constexpr int kStageFloats = kChunk * kKStride;
+constexpr int kRegKeysSmall = 16;                     // keys per lane held in registers
+constexpr int kRegKeysLarge = 40;
 
 struct SelParams {
   const float* qbar;
@@ -32,111 +44,267 @@ struct SelParams {
   int32_t* marg;
   __nv_bfloat16* mask;
   float* logits;
-  int nB, nBpow, nBp, R, k_c, n_neg, m;
+  int nB, nBk, nBp, k_c, n_neg, m;
 };
 
-__device__ __forceinline__ uint64_t rank_key(float l, int j) {
-  if (l == 0.f) l = 0.f;  // -0 and +0 are equal logits
-  uint32_t u = __float_as_uint(l);
-  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-  return (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(0xFFFFFFFFu - static_cast<uint32_t>(j));
+// Larger logit -> larger unsigned key; -0 and +0 map to the same key. Every finite or
+// infinite logit maps to a key >= 1, so 0 marks an empty slot.
+__device__ __forceinline__ uint32_t order_key(float l) {
+  if (l == 0.f) l = 0.f;
+  const uint32_t u = __float_as_uint(l);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_kernel(SelParams p) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  uint64_t* keys = reinterpret_cast<uint64_t*>(smem);                   // [R][nBpow]
-  float* qb = reinterpret_cast<float*>(keys + p.R * p.nBpow);            // [R][128]
-  unsigned char* cls = reinterpret_cast<unsigned char*>(qb + p.R * kHeadDim);  // [R][nBpow]
+// Stage channels [c0, c0+16) of key blocks [jbase, jbase+512) channel-major: a half warp
+// reads one block's 64 contiguous bytes, each lane writes one (channel, block) slot.
+__device__ __forceinline__ void stage_kbar(const float* kb, float* dst, int jbase, int c0, int nB,
+                                           int tid) {
+#pragma unroll 4
+  for (int t = 0; t < kJPass * kChunk / kSelThreads; ++t) {
+    const int e = tid + t * kSelThreads;
+    const int jj = e >> 4, c = e & (kChunk - 1);
+    if (jbase + jj < nB)
+      cp_async4(smem_u32(dst + c * kKStride + jj),
+                kb + static_cast<size_t>(jbase + jj) * kHeadDim + c0 + c);
+  }
+}
 
-  const int i0 = blockIdx.x * p.R, bh = blockIdx.y, tid = threadIdx.x;
-  const int rows = min(p.R, p.nB - i0);
-  const int nB = p.nB, nBpow = p.nBpow;
-
-  for (int x = tid; x < rows * kHeadDim; x += kSelThreads)
-    qb[x] = p.qbar[(static_cast<size_t>(bh) * nB + i0) * kHeadDim + x];
-  __syncthreads();
-
-  // ---- 1. logits
-  for (int j = tid; j < nBpow; j += kSelThreads) {
-    if (j < nB) {
-      float acc[kSelRowsMax];
+// One row's keys for the warp: slot t of lane l is block j = 32*t + l (0 when j >= nB).
+// KPL > 0 keeps them in registers (nB <= 32*KPL); KPL == 0 reads shared memory.
+template <int KPL>
+struct RowKeys {
+  uint32_t v[KPL > 0 ? KPL : 1];
+  const uint32_t* kr;
+  int nB, lane, nt;
+  __device__ __forceinline__ void load(const uint32_t* kr_, int nB_, int nBp, int lane_) {
+    kr = kr_;
+    nB = nB_;
+    lane = lane_;
+    nt = nBp >> 5;
+    if constexpr (KPL > 0) {
 #pragma unroll
-      for (int r = 0; r < kSelRowsMax; ++r) acc[r] = 0.f;
-      const float4* kr = reinterpret_cast<const float4*>(p.kbar + (static_cast<size_t>(bh) * nB + j) * kHeadDim);
-      for (int c4 = 0; c4 < kHeadDim / 4; ++c4) {
-        const float4 kv = kr[c4];
-#pragma unroll
-        for (int r = 0; r < kSelRowsMax; ++r) {
-          if (r < rows) {
-            const float4 qv = reinterpret_cast<const float4*>(qb + r * kHeadDim)[c4];
-            acc[r] = __fadd_rn(acc[r], __fmul_rn(qv.x, kv.x));
-            acc[r] = __fadd_rn(acc[r], __fmul_rn(qv.y, kv.y));
-            acc[r] = __fadd_rn(acc[r], __fmul_rn(qv.z, kv.z));
-            acc[r] = __fadd_rn(acc[r], __fmul_rn(qv.w, kv.w));
-          }
-        }
+      for (int t = 0; t < KPL; ++t) {
+        const int j = 32 * t + lane;
+        v[t] = j < nB ? kr[j] : 0u;
       }
-#pragma unroll
-      for (int r = 0; r < kSelRowsMax; ++r) {
-        if (r < rows) {
-          keys[r * nBpow + j] = rank_key(acc[r], j);
-          if (p.logits) p.logits[(static_cast<size_t>(bh) * nB + i0 + r) * nB + j] = acc[r];
-        }
-      }
-    } else {
-      for (int r = 0; r < rows; ++r) keys[r * nBpow + j] = 0ull;  // below every real key
     }
   }
-  __syncthreads();
+  __device__ __forceinline__ uint32_t at(int t) const {
+    if constexpr (KPL > 0) {
+      return v[t];
+    } else {
+      const int j = 32 * t + lane;
+      return j < nB ? kr[j] : 0u;
+    }
+  }
+};
 
-  // ---- 2. bitonic sort, descending, every row at once (nBpow = 2^lgn)
-  const int lgn = __ffs(nBpow) - 1;
-  const int half = nBpow >> 1;
-  for (int lk = 1; lk <= lgn; ++lk) {
-    for (int lj = lk - 1; lj >= 0; --lj) {
-      const int jj = 1 << lj;
-      for (int x = tid; x < rows * half; x += kSelThreads) {
-        const int r = x >> (lgn - 1), t = x & (half - 1);
-        const int i = ((t >> lj) << (lj + 1)) | (t & (jj - 1));
-        const int l = i + jj;
-        uint64_t* kr = keys + r * nBpow;
-        const uint64_t a = kr[i], b = kr[l];
-        const bool desc = ((i >> lk) & 1) == 0;
-        if (desc ? (a < b) : (a > b)) {
-          kr[i] = b;
-          kr[l] = a;
+template <int KPL, class Pred>
+__device__ __forceinline__ int warp_count(const RowKeys<KPL>& K, Pred pred) {
+  int c = 0;
+  if constexpr (KPL > 0) {
+#pragma unroll
+    for (int t = 0; t < KPL; ++t) c += pred(K.v[t]) ? 1 : 0;
+  } else {
+    for (int t = 0; t < K.nt; ++t) c += pred(K.at(t)) ? 1 : 0;
+  }
+  return __reduce_add_sync(0xffffffffu, c);
+}
+
+// Classify one row and write its lists and mask row (one warp, warp-uniform control).
+template <int KPL>
+__device__ void classify_row(const SelParams& p, const uint32_t* kr, size_t row, int lane) {
+  RowKeys<KPL> K;
+  K.load(kr, p.nB, p.nBp, lane);
+  const int k_c = p.k_c, n_neg = p.n_neg;
+
+  // k_c-th largest key: the largest T with #{key >= T} >= k_c.
+  uint32_t Tc = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = Tc | (1u << bit);
+    const int c = warp_count(K, [cand](uint32_t x) { return x >= cand; });
+    if (c >= k_c) {
+      Tc = cand;
+      if (c == k_c) break;  // {key >= cand} is exactly the critical set
+    }
+  }
+  const int need_c = k_c - warp_count(K, [Tc](uint32_t x) { return x > Tc; });
+
+  // n_neg-th smallest key, searched as the n_neg-th largest complemented key; empty
+  // slots (0) are excluded by testing 1 <= key <= X as (key - 1) < X.
+  uint32_t Tn = 0;
+  int need_n = 0, eq_n = 0;
+  if (n_neg > 0) {
+    uint32_t T = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit), X = ~cand;
+      const int c = warp_count(K, [X](uint32_t x) { return x - 1u < X; });
+      if (c >= n_neg) {
+        T = cand;
+        if (c == n_neg) break;
+      }
+    }
+    Tn = ~T;
+    need_n = n_neg - warp_count(K, [Tn](uint32_t x) { return x - 1u < Tn - 1u; });
+    eq_n = warp_count(K, [Tn](uint32_t x) { return x == Tn; });
+  }
+
+  const unsigned lt = (1u << lane) - 1u;
+  int nc = 0, nm = 0, seen_c = 0, seen_n = 0;
+  auto chunk = [&](int t, uint32_t key) {
+    const int j = 32 * t + lane;
+    const bool valid = j < p.nB;
+    const bool eqc = valid && key == Tc;
+    const unsigned be = __ballot_sync(0xffffffffu, eqc);
+    const bool isc = valid && (key > Tc || (eqc && seen_c + __popc(be & lt) < need_c));
+    seen_c += __popc(be);
+    bool isn = false;
+    if (n_neg > 0) {
+      const bool eqn = valid && key == Tn;
+      const unsigned bn = __ballot_sync(0xffffffffu, eqn);
+      isn = valid && (key < Tn || (eqn && seen_n + __popc(bn & lt) >= eq_n - need_n));
+      seen_n += __popc(bn);
+    }
+    const bool ism = valid && !isc && !isn;
+    const unsigned bc = __ballot_sync(0xffffffffu, isc);
+    const unsigned bm = __ballot_sync(0xffffffffu, ism);
+    // The counts are exact by construction; the bounds only keep a row inside its list.
+    const int pc = nc + __popc(bc & lt), pm = nm + __popc(bm & lt);
+    if (isc && pc < k_c) p.crit[row * k_c + pc] = j;
+    if (ism && pm < p.m) p.marg[row * p.m + pm] = j;
+    nc += __popc(bc);
+    nm += __popc(bm);
+    p.mask[row * p.nBp + j] = __float2bfloat16_rn(ism ? 1.f : 0.f);
+  };
+  if constexpr (KPL > 0) {
+#pragma unroll
+    for (int t = 0; t < KPL; ++t)
+      if (t < K.nt) chunk(t, K.v[t]);
+  } else {
+    for (int t = 0; t < K.nt; ++t) chunk(t, K.at(t));
+  }
+}
+
+template <int RT>
+__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelParams p) {
+  constexpr int R = 2 * RT;
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* qs = reinterpret_cast<float*>(smem);                 // [R][128] row means
+  float* kT = qs + R * kHeadDim;                              // [2][kChunk][kKStride]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(kT + 2 * kStageFloats);  // [R][nBk]
+
+  const int tid = threadIdx.x, bh = blockIdx.y;
+  const int nB = p.nB, i0 = blockIdx.x * R;
+  const int rows = min(R, nB - i0);
+  const float* kb = p.kbar + static_cast<size_t>(bh) * nB * kHeadDim;
+
+  for (int x = tid; x < R * kHeadDim / 4; x += kSelThreads) {
+    const int r = x / (kHeadDim / 4);
+    reinterpret_cast<float4*>(qs)[x] =
+        r < rows ? reinterpret_cast<const float4*>(p.qbar + (static_cast<size_t>(bh) * nB + i0) * kHeadDim)[x]
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+
+  // ---- 1. logits, 512 key blocks per pass
+  const int rg = tid / kGroupThreads, tl = tid % kGroupThreads;
+  const int row0 = rg * RT;
+  for (int jbase = 0; jbase < nB; jbase += kJPass) {
+    float acc[RT][4];
+#pragma unroll
+    for (int r = 0; r < RT; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+    const int j0 = jbase + kJPerThread * tl;
+    const bool active = j0 < nB;
+
+    stage_kbar(kb, kT, jbase, 0, nB, tid);
+    cp_async_commit();
+    for (int s = 0; s < kStages; ++s) {
+      if (s + 1 < kStages) {
+        stage_kbar(kb, kT + ((s + 1) & 1) * kStageFloats, jbase, (s + 1) * kChunk, nB, tid);
+        cp_async_commit();
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();
+      if (active) {
+        // Separate round-to-nearest multiply and add (never contracted into an FMA).
+        const float* kt = kT + (s & 1) * kStageFloats + kJPerThread * tl;
+        const float* qrow = qs + row0 * kHeadDim + s * kChunk;
+#pragma unroll
+        for (int c4 = 0; c4 < kChunk; c4 += 4) {
+          float4 kv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) kv[e] = *reinterpret_cast<const float4*>(kt + (c4 + e) * kKStride);
+#pragma unroll
+          for (int r = 0; r < RT; ++r) {
+            const float4 q = *reinterpret_cast<const float4*>(qrow + r * kHeadDim + c4);
+            const float qc[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {  // channel c4 + e, in order
+              acc[r][0] = __fadd_rn(acc[r][0], __fmul_rn(qc[e], kv[e].x));
+              acc[r][1] = __fadd_rn(acc[r][1], __fmul_rn(qc[e], kv[e].y));
+              acc[r][2] = __fadd_rn(acc[r][2], __fmul_rn(qc[e], kv[e].z));
+              acc[r][3] = __fadd_rn(acc[r][3], __fmul_rn(qc[e], kv[e].w));
+            }
+          }
         }
       }
       __syncthreads();
     }
-  }
 
-  // ---- 3. classes by sorted position, then ascending compaction
-  for (int r = 0; r < rows; ++r) {
-    for (int pos = tid; pos < nB; pos += kSelThreads) {
-      const int j = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(keys[r * nBpow + pos]));
-      cls[r * nBpow + j] = pos < p.k_c ? 0 : (pos < nB - p.n_neg ? 1 : 2);
+    if (active) {
+#pragma unroll
+      for (int r = 0; r < RT; ++r) {
+        const int row = row0 + r;
+        if (row < rows) {
+          const float* l = acc[r];
+          uint4 kv;
+          kv.x = order_key(l[0]);
+          kv.y = j0 + 1 < nB ? order_key(l[1]) : 0u;
+          kv.z = j0 + 2 < nB ? order_key(l[2]) : 0u;
+          kv.w = j0 + 3 < nB ? order_key(l[3]) : 0u;
+          *reinterpret_cast<uint4*>(keys + row * p.nBk + j0) = kv;
+          if (p.logits) {
+            float* lr = p.logits + (static_cast<size_t>(bh) * nB + i0 + row) * nB;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (j0 + e < nB) lr[j0 + e] = l[e];
+          }
+        }
+      }
     }
   }
   __syncthreads();
 
+  // ---- 2-3. thresholds and lists, one warp per row
   const int warp = tid >> 5, lane = tid & 31;
-  const unsigned lt = (1u << lane) - 1u;
   for (int r = warp; r < rows; r += kSelThreads / 32) {
     const size_t row = static_cast<size_t>(bh) * nB + i0 + r;
-    int nc = 0, nm = 0;
-    for (int base = 0; base < p.nBp; base += 32) {
-      const int j = base + lane;
-      const int c = j < nB ? cls[r * nBpow + j] : 3;
-      const unsigned bc = __ballot_sync(0xffffffffu, c == 0);
-      const unsigned bm = __ballot_sync(0xffffffffu, c == 1);
-      if (c == 0) p.crit[row * p.k_c + nc + __popc(bc & lt)] = j;
-      if (c == 1) p.marg[row * p.m + nm + __popc(bm & lt)] = j;
-      nc += __popc(bc);
-      nm += __popc(bm);
-      p.mask[row * p.nBp + j] = __float2bfloat16_rn(c == 1 ? 1.f : 0.f);
-    }
+    const uint32_t* kr = keys + r * p.nBk;
+    if (p.nBp <= 32 * kRegKeysSmall)
+      classify_row<kRegKeysSmall>(p, kr, row, lane);
+    else if (p.nBp <= 32 * kRegKeysLarge)
+      classify_row<kRegKeysLarge>(p, kr, row, lane);
+    else
+      classify_row<0>(p, kr, row, lane);
   }
+}
+
+template <int RT>
+cudaError_t launch_rt(const Dims& g, const SelParams& p, cudaStream_t st) {
+  constexpr int R = 2 * RT;
+  const size_t smem = static_cast<size_t>(R) * kHeadDim * 4 +
+                      static_cast<size_t>(2) * kStageFloats * 4 +
+                      static_cast<size_t>(R) * p.nBk * 4;
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<RT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  {
+    TraceScope ts_("select_kernel", st);
+    select_kernel<RT><<<dim3((g.nB + R - 1) / R, g.BH), kSelThreads, smem, st>>>(p);
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -144,12 +312,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelParams p) {
 cudaError_t launch_select(const Dims& g, const float* q_bar, const float* k_bar, int k_c,
                           int n_neg, int m, int32_t* crit, int32_t* marg, void* mask,
                           float* logits, cudaStream_t st) {
-  int nBpow = 1;
-  while (nBpow < g.nB) nBpow <<= 1;
-  if (nBpow < 2) nBpow = 2;
-  int R = kSelKeys / nBpow;
-  if (R > kSelRowsMax) R = kSelRowsMax;
-  if (R < 1) return cudaErrorInvalidValue;
   SelParams p;
   p.qbar = q_bar;
   p.kbar = k_bar;
@@ -158,22 +320,17 @@ cudaError_t launch_select(const Dims& g, const float* q_bar, const float* k_bar,
   p.mask = static_cast<__nv_bfloat16*>(mask);
   p.logits = logits;
   p.nB = g.nB;
-  p.nBpow = nBpow;
+  p.nBk = (g.nB + 3) & ~3;
   p.nBp = g.nBp;
-  p.R = R;
   p.k_c = k_c;
   p.n_neg = n_neg;
   p.m = m;
-  const size_t smem = static_cast<size_t>(R) * nBpow * 8 + static_cast<size_t>(R) * kHeadDim * 4 +
-                      static_cast<size_t>(R) * nBpow;
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  {
-    TraceScope ts_("select_kernel", st);
-    select_kernel<<<dim3((g.nB + R - 1) / R, g.BH), kSelThreads, smem, st>>>(p);
-  }
-  return cudaGetLastError();
+  // Rows per CTA shrink with nB so that the keys of all rows fit in shared memory
+  // (R * nBk * 4 bytes <= 128 KB).
+  if (g.nB <= 2048) return launch_rt<8>(g, p, st);
+  if (g.nB <= 4096) return launch_rt<4>(g, p, st);
+  if (g.nB <= 8192) return launch_rt<2>(g, p, st);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace sgs

@@ -55,6 +55,25 @@ def run_gpu(q, k, v, rho, nu, logits=True, repeat=1):
     return res
 
 
+def run_gpu_select(q, k, v, rho, nu):
+    """Run prepare and select only (logits kept); return CPU numpy copies."""
+    ensure_lib()
+    B, H, N, d = q.shape
+    qd, kd, vd = (t.cuda().contiguous() for t in (q, k, v))
+    ws = S.alloc_workspace(B, H, N, qd.device)
+    p = S.sagesla_prepare(qd, kd, vd, ws)
+    s = S.sagesla_select(p.q_bar, p.k_bar, N, rho, nu, logits=True)
+    torch.cuda.synchronize()
+    S.sagesla_check_status(ws)
+    return dict(
+        q8=p.q8.cpu().numpy(), k8=p.k8.cpu().numpy(), q_scale=p.q_scale.cpu().numpy(),
+        k_scale=p.k_scale.cpu().numpy(), k_mean=p.k_mean.cpu().numpy(),
+        q_bar=p.q_bar.cpu().numpy(), k_bar=p.k_bar.cpu().numpy(),
+        crit=s.crit.cpu().numpy(), marg=s.marg.cpu().numpy()[..., : s.m],
+        mask=s.mask.float().cpu().numpy(), k_c=s.k_c, n_neg=s.n_neg, m=s.m,
+        logits=s.logits.cpu().numpy())
+
+
 def bits(a):
     return np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
 
@@ -87,6 +106,12 @@ def compare_lists(g, sel, heads=slice(None)):
         np.testing.assert_array_equal(bits(g["logits"][:, heads]), bits(sel.logits))
     bad = np.argwhere((gc != sel.crit).any(-1) | ((gm != sel.marg).any(-1) if sel.m else False))
     nB = sel.logits.shape[-1]
+    # the bf16 marginal mask: 1 exactly on the marginal blocks, 0 elsewhere and on padding
+    gmask = g["mask"][:, heads]
+    ok_rows = np.ones(gmask.shape[:-1], dtype=bool)
+    ok_rows[tuple(bad.T)] = False
+    np.testing.assert_array_equal(gmask[..., :nB][ok_rows], sel.marg_mask()[ok_rows])
+    assert not gmask[..., nB:].any()
     near = 0
     for idx in bad:
         idx = tuple(idx)

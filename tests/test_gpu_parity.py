@@ -12,7 +12,8 @@ import torch
 import oracle as O
 from quantized_block_sparse_b200.inputs import WORKLOADS, make_qkv, make_random_qkv, sweep_workload
 from tests.gpu_helpers import (assert_linear_states_close, assert_output_close,
-                               assert_prepare_bitexact, compare_lists, f32, run_gpu)
+                               assert_prepare_bitexact, compare_lists, f32, run_gpu,
+                               run_gpu_select)
 
 pytestmark = pytest.mark.gpu
 
@@ -135,3 +136,16 @@ def test_720p_full_size_sampled():
 def test_sweep_full_size_sampled(rho):
     near, res = _sampled_check(sweep_workload(rho), heads_for_oracle=1, qblocks_per_head=8, seed=1)
     assert near == 0
+
+
+@pytest.mark.parametrize("N", [90000, 140000, 270000])
+def test_select_large_block_counts(N):
+    # nB = 1407: row keys read from shared memory instead of registers; nB = 2188 and
+    # 4219: 8 and 4 query-block rows per CTA. Prepare and select only.
+    q, k, v = make_random_qkv(1, 1, N, seed=N)
+    g = run_gpu_select(q, k, v, 0.1, 0.45)
+    prep = O.prepare(f32(q), f32(k))
+    sel = O.select(prep.q_bar, prep.k_bar, 0.1, 0.45)
+    assert_prepare_bitexact(g, prep)
+    assert (g["k_c"], g["n_neg"], g["m"]) == (sel.k_c, sel.n_neg, sel.m)
+    assert compare_lists(g, sel) == 0
