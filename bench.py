@@ -129,7 +129,7 @@ def oracle_sample(q, k, v, wl, n_small=None, n_large=None):
 
 def run_reference(args, wl):
     """`--impl reference`: the CPU oracle, as it stands, on a bounded sample per step."""
-    rank = int(os.environ.get("RANK", "0"))
+    rank, _, _ = rank_env()
     if rank != 0:
         return 0
     q, k, v = make_workload_qkv(wl)
@@ -211,6 +211,43 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------------------ ranks
+# One process per GPU (torchrun). The path has no exchange step: every rank runs an
+# independent replica of the workload; ranks meet only for barriers around the timed
+# region and for the max of the per-rank times.
+def rank_env():
+    """(rank, world, local_rank) from the torchrun environment (1 process without it)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_ranks(world: int, backend: str, device=None, timeout_s: float = 120.0):
+    """Process group for world > 1 (short timeout so a missing rank ends with an error)."""
+    if world <= 1:
+        return
+    import datetime
+
+    import torch.distributed as dist
+    kw = {"device_id": device} if backend == "nccl" else {}
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+
+def max_over_ranks_of(x: float, world: int, device=None) -> float:
+    """The largest per-rank value (the job's step time is its slowest rank's)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tops(ops_per_rank: float, world: int, step_ms: float) -> float:
+    """Throughput of the whole job: the work of all ranks over the slowest rank's time."""
+    return ops_per_rank * world / (step_ms * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_ours(args, wl):
     import torch
@@ -218,26 +255,17 @@ def run_ours(args, wl):
 
     from quantized_block_sparse_b200 import sagesla as S
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = rank_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+    init_ranks(world, "nccl", dev)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks_of(x, world, dev)
 
     S.lib()
     q, k, v = make_workload_qkv(wl)
@@ -317,11 +345,10 @@ def run_ours(args, wl):
     att_ms = kern.get("attn_kernel", {}).get("avg_ms", float("nan"))
     achieved = bf16_equiv / (att_ms * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
-    dense_ops = dense_equiv_ops(wl) * world
 
     line = {
         "metric": METRIC,
-        "value": dense_ops / (step_ms * 1e-3) / 1e12,
+        "value": whole_job_tops(dense_equiv_ops(wl), world, step_ms),
         "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_ms,
@@ -339,7 +366,7 @@ def run_ours(args, wl):
                               f"{pairs} executed 64x64 block pairs; peak = {peak_src} cuBLAS bf16 burst; "
                               f"traffic = DRAM bytes per launch from the committed ncu summary "
                               f"(null once the kernel source differs from the profiled one)")},
-        "e2e": {"value": dense_ops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+        "e2e": {"value": whole_job_tops(dense_equiv_ops(wl), world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(round(launches_per_step * args.steps)),
         "clocks": clk,

@@ -107,6 +107,22 @@ __device__ __forceinline__ int quant_code(float x, float s) {
   return max(-127, min(127, c));
 }
 
+// The same code byte as quant_code(x, s) (rint(fl32(x/s)), clamped), without a division on
+// the common path. With rs = fl32(1/s) and y = fl32(x*rs): |x/s| <= 127*(1+2^-23) because
+// s = fl32(amax/127), so |y - x/s| < 1.6e-5 and |y - fl32(x/s)| < 2e-5. Unless y lies within
+// 3e-5 of a half-integer, y and fl32(x/s) round to the same integer; those rare elements take
+// the exact division. rint is done by adding 1.5*2^23 (exact for |y| < 2^22): the low byte
+// of the sum's bit pattern is then the two's-complement code, and |rint(y)| <= 127 needs no
+// clamp. Returns the byte in bits 0-7.
+constexpr float kRintMagic = 12582912.f;  // 1.5 * 2^23
+__device__ __forceinline__ uint32_t quant_byte(float x, float s, float rs) {
+  const float y = __fmul_rn(x, rs);
+  const float t = __fadd_rn(y, kRintMagic);
+  const float e = __fsub_rn(__fsub_rn(t, kRintMagic), y);  // rint(y) - y, exact
+  if (fabsf(e) > 0.49997f) return static_cast<uint32_t>(quant_code(x, s)) & 0xffu;
+  return __float_as_uint(t) & 0xffu;
+}
+
 __device__ __forceinline__ void unpack8(const uint4 u, float (&f)[8]) {
   const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
@@ -117,7 +133,9 @@ __device__ __forceinline__ void unpack8(const uint4 u, float (&f)[8]) {
   }
 }
 
-__device__ __forceinline__ float phi_f32(float x) { return x > 0.f ? __fadd_rn(x, 1.f) : expf(x); }
+// phi feeds bf16 MMA operands and the fp32 z sums, so the fast exponential (relative error
+// ~2^-21, far below the bf16 rounding of phi) is enough.
+__device__ __forceinline__ float phi_f32(float x) { return x > 0.f ? __fadd_rn(x, 1.f) : __expf(x); }
 
 // One CTA per (head, 64-token block). All three input blocks are requested at once (two
 // bulk copies for the raw Q and K rows, two TMA boxes for V straight into the MN-major
@@ -183,6 +201,9 @@ __global__ void __launch_bounds__(kPrepThreads, 3) prep_block_kernel(const __gri
   }
   const float2 amax = block_max2(lq, lk, red);
   const float sq = __fdiv_rn(amax.x, 127.f), sk = __fdiv_rn(amax.y, 127.f);
+  // fast path only for a normal, finite reciprocal; otherwise every element divides exactly
+  const float rq = __frcp_rn(sq), rk = __frcp_rn(sk);
+  const bool fast = sq > 1e-30f && sk > 1e-30f && rq < 1e30f && rk < 1e30f;
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk) {
     const int r = rg + 16 * kk;
@@ -191,10 +212,18 @@ __global__ void __launch_bounds__(kPrepThreads, 3) prep_block_kernel(const __gri
       float fq[8], fk[8];
       unpack8(*reinterpret_cast<const uint4*>(sQ + r * kHeadDim + 8 * chunk), fq);
       unpack8(*reinterpret_cast<const uint4*>(sK + r * kHeadDim + 8 * chunk), fk);
+      if (fast) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        cq[e >> 2] |= (static_cast<uint32_t>(quant_code(__fmul_rn(fq[e], p.c_s), sq)) & 0xffu) << (8 * (e & 3));
-        ck[e >> 2] |= (static_cast<uint32_t>(quant_code(__fsub_rn(fk[e], mu8[e]), sk)) & 0xffu) << (8 * (e & 3));
+        for (int e = 0; e < 8; ++e) {
+          cq[e >> 2] |= quant_byte(__fmul_rn(fq[e], p.c_s), sq, rq) << (8 * (e & 3));
+          ck[e >> 2] |= quant_byte(__fsub_rn(fk[e], mu8[e]), sk, rk) << (8 * (e & 3));
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          cq[e >> 2] |= (static_cast<uint32_t>(quant_code(__fmul_rn(fq[e], p.c_s), sq)) & 0xffu) << (8 * (e & 3));
+          ck[e >> 2] |= (static_cast<uint32_t>(quant_code(__fsub_rn(fk[e], mu8[e]), sk)) & 0xffu) << (8 * (e & 3));
+        }
       }
     }
     *reinterpret_cast<uint2*>(p.q8 + (prow0 + r) * kHeadDim + 8 * chunk) = make_uint2(cq[0], cq[1]);
