@@ -180,19 +180,24 @@ __global__ void __launch_bounds__(256) zsum_kernel(const float* __restrict__ z,
 }
 
 // ------------------------------------------------------------------ O_l
-constexpr int kLinSmem = 32768 + 65536 + 1024 + 256;
+// One CTA per pair of query blocks, 256 threads: thread t builds phi(Q~) for row t%128 and
+// channels [64*(t/128), +64) and its part of the denominator; eight warps then read the two
+// 128x128 products back, each a quadrant of rows and half of the columns.
+constexpr int kLinThreads = 256;
+constexpr int kLinSmem = 32768 + 65536 + 1024 + 1024 + 256;
 
-__global__ void __launch_bounds__(128) linout_kernel(const __grid_constant__ CUtensorMap tmH,
-                                                     const __nv_bfloat16* __restrict__ q,
-                                                     const float* __restrict__ Z, float c_s,
-                                                     __nv_bfloat16* __restrict__ Ol, int N,
-                                                     int nB, int* status) {
+__global__ void __launch_bounds__(kLinThreads) linout_kernel(const __grid_constant__ CUtensorMap tmH,
+                                                             const __nv_bfloat16* __restrict__ q,
+                                                             const float* __restrict__ Z, float c_s,
+                                                             __nv_bfloat16* __restrict__ Ol, int N,
+                                                             int nB, int* status) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   unsigned char* sA = smem;            // phi(Q~): 2 column blocks x 128 rows x 128 B
   unsigned char* sH = smem + 32768;    // H_i0, H_i1: each 2 e-groups x 128 c rows x 128 B
-  uint64_t* hfull = reinterpret_cast<uint64_t*>(smem + 32768 + 65536);
+  float* dpart = reinterpret_cast<float*>(smem + 32768 + 65536);  // [2][128] denominator halves
+  uint64_t* hfull = reinterpret_cast<uint64_t*>(smem + 32768 + 65536 + 1024);
   uint64_t* mdone = hfull + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + 1);
   __shared__ int abort_flag;
@@ -221,38 +226,42 @@ __global__ void __launch_bounds__(128) linout_kernel(const __grid_constant__ CUt
     }
   }
 
-  // phi(Q~) row r and its denominator phi(Q~).Z_i (with the bf16-rounded phi values the
-  // tensor core sees).
-  const int r = tid;
-  const int i = i0 + (r >> 6);
-  const int t = i * 64 + (r & 63);
-  const bool valid = (i < nB) && (t < N);
-  float den = 1.f;
+  // phi(Q~) for (row r, 64 channels) and that part of phi(Q~).Z_i, with the bf16-rounded
+  // phi values the tensor core sees. phi is rounded to bf16, so the fast exponential
+  // (relative error ~2^-21) is enough.
   {
-    const __nv_bfloat16* qr = q + (static_cast<size_t>(bh) * N + (valid ? t : 0)) * kHeadDim;
-    const float* zr = Z + (static_cast<size_t>(bh) * nB + (i < nB ? i : 0)) * kHeadDim;
+    const int r = tid & 127, chh = tid >> 7;
+    const int i = i0 + (r >> 6);
+    const int t = i * 64 + (r & 63);
+    const bool valid = (i < nB) && (t < N);
+    const __nv_bfloat16* qr = q + (static_cast<size_t>(bh) * N + (valid ? t : 0)) * kHeadDim + 64 * chh;
+    const float* zr = Z + (static_cast<size_t>(bh) * nB + (i < nB ? i : 0)) * kHeadDim + 64 * chh;
     float dacc = 0.f;
 #pragma unroll
-    for (int cb = 0; cb < 16; ++cb) {  // 8 channels per chunk
+    for (int cb = 0; cb < 8; ++cb) {  // 8 channels per chunk
       uint32_t w[4] = {0, 0, 0, 0};
       if (valid) {
         const uint4 u = *reinterpret_cast<const uint4*>(qr + 8 * cb);
+        const float4 z0 = *reinterpret_cast<const float4*>(zr + 8 * cb);
+        const float4 z1 = *reinterpret_cast<const float4*>(zr + 8 * cb + 4);
+        const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
         const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = __bfloat1622float2(b2[e]);
           const float x0 = __fmul_rn(f.x, c_s), x1 = __fmul_rn(f.y, c_s);
-          const float p0 = x0 > 0.f ? x0 + 1.f : expf(x0);
-          const float p1 = x1 > 0.f ? x1 + 1.f : expf(x1);
+          const float p0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
+          const float p1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
           w[e] = pack_bf16x2(p0, p1);
           const float2 pr2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
-          dacc = fmaf(pr2.x, zr[8 * cb + 2 * e], dacc);
-          dacc = fmaf(pr2.y, zr[8 * cb + 2 * e + 1], dacc);
+          dacc = fmaf(pr2.x, zz[2 * e], dacc);
+          dacc = fmaf(pr2.y, zz[2 * e + 1], dacc);
         }
       }
-      st_shared_v4(smem_u32(sA) + (cb >> 3) * 16384 + sw128_offset(r, cb & 7), w[0], w[1], w[2], w[3]);
+      const int cg = 8 * chh + cb;  // 16-byte chunk index over the 128 channels
+      st_shared_v4(smem_u32(sA) + (cg >> 3) * 16384 + sw128_offset(r, cg & 7), w[0], w[1], w[2], w[3]);
     }
-    if (valid) den = dacc;
+    dpart[chh * 128 + r] = dacc;
   }
   fence_async_smem();
   tc_fence_before();
@@ -272,20 +281,30 @@ __global__ void __launch_bounds__(128) linout_kernel(const __grid_constant__ CUt
           mma_bf16(taddr + 128 * b, a, bd, idesc, kk > 0);
         }
       }
+    } else {
+      mbar_wait_inflight(smem_u32(hfull), 0, status);
     }
     mma_commit(smem_u32(mdone));
   }
   __syncwarp();
   const bool ok = mbar_wait(smem_u32(mdone), 0, &abort_flag, status);
   tc_fence_after();
-  if (ok && (i < nB)) {  // warp-uniform: rows 0-63 -> warps 0,1; rows 64-127 -> warps 2,3
-    const int half = warp >> 1;
-    const float inv = 1.f / den;
-    __nv_bfloat16* dst = Ol + (static_cast<size_t>(bh) * N + (valid ? t : 0)) * kHeadDim;
+  // Warp w: TMEM lane quadrant w%4 (rows 32*(w%4) ..), output columns [64*(w/4), +64).
+  // Rows 0-63 (block i0) read the product with H_i0 (columns 0-127), rows 64-127 the one
+  // with H_i0+1 (columns 128-255).
+  const int wq = warp & 3, ch2 = warp >> 2;
+  const int r = 32 * wq + lane;
+  const int half = wq >> 1;
+  const int i = i0 + half;
+  const int t = i * 64 + (r & 63);
+  const bool valid = (i < nB) && (t < N);
+  if (ok && (i < nB)) {  // warp-uniform
+    const float inv = 1.f / (dpart[r] + dpart[128 + r]);
+    __nv_bfloat16* dst = Ol + (static_cast<size_t>(bh) * N + (valid ? t : 0)) * kHeadDim + 64 * ch2;
 #pragma unroll
-    for (int cchunk = 0; cchunk < 4; ++cchunk) {
+    for (int cchunk = 0; cchunk < 2; ++cchunk) {
       uint32_t rr[32];
-      tmem_ld32_sync(taddr + (static_cast<uint32_t>(32 * warp) << 16) + 128 * half + 32 * cchunk, rr);
+      tmem_ld32_sync(taddr + (static_cast<uint32_t>(32 * wq) << 16) + 128 * half + 64 * ch2 + 32 * cchunk, rr);
       if (valid) {
         uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cchunk);
 #pragma unroll
@@ -342,7 +361,7 @@ cudaError_t launch_linear(const Dims& g, const void* q, float sm_scale, const vo
   }
   {
     TraceScope ts_("linout_kernel", st);
-    linout_kernel<<<dim3((g.nB + 1) / 2, g.BH), 128, kLinSmem, st>>>(
+    linout_kernel<<<dim3((g.nB + 1) / 2, g.BH), kLinThreads, kLinSmem, st>>>(
       tmH, static_cast<const __nv_bfloat16*>(q), Zbuf, sm_scale, Ol, g.N, g.nB, status);
   }
   return cudaGetLastError();
