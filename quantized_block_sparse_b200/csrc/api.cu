@@ -26,6 +26,8 @@ WsLayout ws_layout(const Dims& g) {
   off = align256(off + static_cast<size_t>(g.BH) * g.nB * kHeadDim * kHeadDim * 2);
   L.Zbuf = off;
   off = align256(off + static_cast<size_t>(g.BH) * g.nB * kHeadDim * 4);
+  L.Zb = off;
+  off = align256(off + static_cast<size_t>(g.BH) * g.nB * kHeadDim * 2);
   L.Ol = off;
   off = align256(off + static_cast<size_t>(g.BH) * g.N * kHeadDim * 2);
   L.total = off;

@@ -11,7 +11,8 @@
 //   hgemm_kernel   H = M . h per head, M the 0/1 marginal mask [nB x nBp] and h viewed as
 //                  [nB x d*d]: a tcgen05 bf16 GEMM (fp32 accumulation in TMEM), 128x128
 //                  output tiles, TMA-fed 3-stage pipeline, bf16 output.
-//   zsum_kernel    Z_i = sum of z_j over the marginal blocks (mask row), fp32, ascending j.
+//   zb_kernel      z_j rounded to bf16; hgemm_kernel's extra column tile gives Z = M . z
+//                  (bf16 operands, fp32 accumulation and output, like H).
 //   linout_kernel  per pair of query blocks: phi(Q~) (recomputed from Q, bf16) times H_i
 //                  on tcgen05 (M = 128 rows = both blocks, one MMA chain per block),
 //                  divided by phi(Q~) . Z_i; bf16 O_l for the attention epilogue.
@@ -22,25 +23,36 @@ namespace sgs {
 namespace {
 
 // ------------------------------------------------------------------ H = M . h
+// Persistent tcgen05 GEMM: each CTA walks output tiles (128 query blocks x 128 columns of
+// h's d*d, N fastest so consecutive tiles share the mask tile in L2). Warp 0 streams A/B
+// k-blocks through a 3-stage ring with TMA, warp 1 issues the MMAs into one of two TMEM
+// accumulators, warps 2-5 drain the other accumulator (bf16) while the next tile runs.
+// One more column tile per row block computes Z = M . z from z rounded to bf16 (the same
+// operand precision as h) and is written in fp32.
 constexpr int kGemmStages = 3;
 constexpr int kGemmStageBytes = 16384 + 16384;
+constexpr int kGemmThreads = 192;
 constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + 1024 + 256;
 
-__global__ void __launch_bounds__(128) hgemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                                                    const __grid_constant__ CUtensorMap tmB,
-                                                    __nv_bfloat16* __restrict__ Hout, int nB,
-                                                    int* status) {
+__global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                                                             const __grid_constant__ CUtensorMap tmB,
+                                                             const __grid_constant__ CUtensorMap tmZ,
+                                                             __nv_bfloat16* __restrict__ Hout,
+                                                             float* __restrict__ Zout, int nB,
+                                                             int n_mt, int n_tiles, int* status) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemmStages * kGemmStageBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + kGemmStages;
-  uint64_t* done = bars + 2 * kGemmStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* tfull = bars + 2 * kGemmStages;   // [2] accumulator ready
+  uint64_t* tempty = tfull + 2;               // [2] accumulator drained
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   __shared__ int abort_flag;
 
-  const int nt = blockIdx.x, mt = blockIdx.y, bh = blockIdx.z;
+  constexpr int kNTH = kHeadDim * kHeadDim / 128;  // 128 N-tiles of H
+  constexpr int kNT = kNTH + 1;                     // + the Z tile
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nK = (nB + 63) / 64;
 
@@ -50,132 +62,140 @@ __global__ void __launch_bounds__(128) hgemm_kernel(const __grid_constant__ CUte
       mbar_init(smem_u32(full + s), 1);
       mbar_init(smem_u32(empty + s), 1);
     }
-    mbar_init(smem_u32(done), 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(tfull + a), 1);
+      mbar_init(smem_u32(tempty + a), 128);
+    }
     fence_mbar_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmZ);
   }
-  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 128);
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 256);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t taddr = *tmem_slot;
 
-  if (warp == 0 && lane == 0) {
-    for (int kb = 0; kb < nK; ++kb) {
-      const int s = kb % kGemmStages;
-      if (kb >= kGemmStages &&
-          !mbar_wait(smem_u32(empty + s), ((kb / kGemmStages) - 1) & 1, &abort_flag, status))
-        break;
-      const uint32_t sa = smem_u32(smem + s * kGemmStageBytes);
-      const uint32_t sb = sa + 16384;
-      mbar_expect_tx(smem_u32(full + s), kGemmStageBytes);
-      tma_load_3d(sa, &tmA, smem_u32(full + s), kb * 64, mt * 128, bh);
-      tma_load_3d(sb, &tmB, smem_u32(full + s), nt * 128, kb * 64, bh);
-      tma_load_3d(sb + 8192, &tmB, smem_u32(full + s), nt * 128 + 64, kb * 64, bh);
-    }
-  } else if (warp == 1 && lane == 0) {
-    constexpr uint32_t idesc = make_idesc(1, 1, 0, 1, 128, 128);
-    bool ok = true;
-    for (int kb = 0; kb < nK && ok; ++kb) {
-      const int s = kb % kGemmStages;
-      ok = mbar_wait(smem_u32(full + s), (kb / kGemmStages) & 1, &abort_flag, status);
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t sa = smem_u32(smem + s * kGemmStageBytes);
-      const uint32_t sb = sa + 16384;
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(taddr, make_sdesc(sa + kk * 32, 16, 1024), make_sdesc(sb + kk * 2048, 8192, 1024),
-                 idesc, (kb | kk) != 0);
-      mma_commit(smem_u32(empty + s));
-    }
-    mma_commit(smem_u32(done));
-  }
-  __syncwarp();
-  const bool ok = mbar_wait(smem_u32(done), 0, &abort_flag, status);
-  tc_fence_after();
-  if (ok) {
-    const int i = mt * 128 + 32 * warp + lane;
-    __nv_bfloat16* dst = Hout + (static_cast<size_t>(bh) * nB + i) * (kHeadDim * kHeadDim) + nt * 128;
-#pragma unroll
-    for (int cchunk = 0; cchunk < 4; ++cchunk) {
-      uint32_t r[32];
-      tmem_ld32_sync(taddr + (static_cast<uint32_t>(32 * warp) << 16) + 32 * cchunk, r);
-      if (i < nB) {
-        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cchunk);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          d4[q] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
-                             pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
-                             pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
-                             pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;  // k-block counter across tiles (ring position)
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+        const int nt = tile % kNT, mt = (tile / kNT) % n_mt, bh = tile / (kNT * n_mt);
+        for (int kb = 0; kb < nK; ++kb, ++it) {
+          const int s = it % kGemmStages;
+          if (it >= kGemmStages &&
+              !mbar_wait(smem_u32(empty + s), ((it / kGemmStages) - 1) & 1, &abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = smem_u32(smem + s * kGemmStageBytes);
+          const uint32_t sb = sa + 16384;
+          mbar_expect_tx(smem_u32(full + s), kGemmStageBytes);
+          tma_load_3d(sa, &tmA, smem_u32(full + s), kb * 64, mt * 128, bh);
+          if (nt < kNTH) {
+            tma_load_3d(sb, &tmB, smem_u32(full + s), nt * 128, kb * 64, bh);
+            tma_load_3d(sb + 8192, &tmB, smem_u32(full + s), nt * 128 + 64, kb * 64, bh);
+          } else {
+            tma_load_3d(sb, &tmZ, smem_u32(full + s), 0, kb * 64, bh);
+            tma_load_3d(sb + 8192, &tmZ, smem_u32(full + s), 64, kb * 64, bh);
+          }
+        }
       }
+      // copies still in flight land before the CTA exits
+      for (int u = max(0, it - kGemmStages); u < it; ++u)
+        mbar_wait_inflight(smem_u32(full + (u % kGemmStages)), (u / kGemmStages) & 1, status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc(1, 1, 0, 1, 128, 128);
+      int it = 0, lt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++lt) {
+        const int a = lt & 1;
+        if (lt >= 2 && !mbar_wait(smem_u32(tempty + a), ((lt >> 1) - 1) & 1, &abort_flag, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < nK; ++kb, ++it) {
+          const int s = it % kGemmStages;
+          if (!mbar_wait(smem_u32(full + s), (it / kGemmStages) & 1, &abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * kGemmStageBytes);
+          const uint32_t sb = sa + 16384;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(taddr + 128 * a, make_sdesc(sa + kk * 32, 16, 1024),
+                     make_sdesc(sb + kk * 2048, 8192, 1024), idesc, (kb | kk) != 0);
+          mma_commit(smem_u32(empty + s));
+        }
+        if (ok) mma_commit(smem_u32(tfull + a));
+      }
+      // every MMA issued completes before the CTA releases TMEM (the last empty commit)
+      if (it > 0) mbar_wait_inflight(smem_u32(empty + ((it - 1) % kGemmStages)), ((it - 1) / kGemmStages) & 1, status);
+    }
+  } else {
+    // epilogue warps 2-5: TMEM lane quadrant w%4 -> rows 32*(w%4) .. of the tile
+    const int wq = warp & 3;
+    int lt = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++lt) {
+      const int a = lt & 1;
+      const int nt = tile % kNT, mt = (tile / kNT) % n_mt, bh = tile / (kNT * n_mt);
+      const bool ok = mbar_wait(smem_u32(tfull + a), (lt >> 1) & 1, &abort_flag, status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int i = mt * 128 + 32 * wq + lane;
+      if (nt < kNTH) {
+        __nv_bfloat16* dst = Hout + (static_cast<size_t>(bh) * nB + i) * (kHeadDim * kHeadDim) + nt * 128;
+#pragma unroll
+        for (int cchunk = 0; cchunk < 4; ++cchunk) {
+          uint32_t r[32];
+          tmem_ld32_sync(taddr + (static_cast<uint32_t>(32 * wq) << 16) + 128 * a + 32 * cchunk, r);
+          if (i < nB) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cchunk);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              d4[q] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
+                                 pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
+                                 pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
+                                 pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+          }
+        }
+      } else {
+        float* dst = Zout + (static_cast<size_t>(bh) * nB + i) * kHeadDim;
+#pragma unroll
+        for (int cchunk = 0; cchunk < 4; ++cchunk) {
+          uint32_t r[32];
+          tmem_ld32_sync(taddr + (static_cast<uint32_t>(32 * wq) << 16) + 128 * a + 32 * cchunk, r);
+          if (i < nB) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cchunk);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) d4[q] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(tempty + a));
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(taddr, 128);
+  if (warp == 1) tmem_dealloc(taddr, 256);
 }
 
-// ------------------------------------------------------------------ Z_i
-// Z_i = sum over j of mask_ij * z_j, ascending j, one fp32 FMA per term (mask_ij is 0 or 1,
-// so each step adds z_j exactly once or leaves the sum unchanged). A CTA covers 16 query
-// blocks; z and the mask rows are staged in shared memory 128 key blocks at a time, so each
-// z row is read from L2 once per 16 query blocks instead of once per query block.
-constexpr int kZRows = 16;
-constexpr int kZChunk = 128;
-constexpr int kZSmem = (kZChunk * kHeadDim + kZRows * kZChunk) * 4;
-
-__global__ void __launch_bounds__(256) zsum_kernel(const float* __restrict__ z,
-                                                   const __nv_bfloat16* __restrict__ mask,
-                                                   float* __restrict__ Z, int nB, int nBp) {
-  extern __shared__ float zsm[];
-  float* zs = zsm;                          // [kZChunk][128]
-  float* ms = zsm + kZChunk * kHeadDim;     // [kZRows][kZChunk]
-  const int i0 = blockIdx.x * kZRows, bh = blockIdx.y, tid = threadIdx.x;
-  const int g = tid >> 7, c = tid & 127;
-  const int rows = min(kZRows, nB - i0);
-  const float* zh = z + static_cast<size_t>(bh) * nB * kHeadDim;
-  const __nv_bfloat16* mh = mask + (static_cast<size_t>(bh) * nB + i0) * nBp;
-  float acc[kZRows / 2];
-#pragma unroll
-  for (int r = 0; r < kZRows / 2; ++r) acc[r] = 0.f;
-
-  for (int j0 = 0; j0 < nB; j0 += kZChunk) {
-    const int jn = min(kZChunk, nB - j0), jn4 = (jn + 3) & ~3;
-    __syncthreads();
-    const float4* src = reinterpret_cast<const float4*>(zh + static_cast<size_t>(j0) * kHeadDim);
-    for (int x = tid; x < jn * (kHeadDim / 4); x += 256) cp_async16(smem_u32(zs + 4 * x), src + x);
-    cp_async_commit();
-    for (int x = jn * (kHeadDim / 4) + tid; x < jn4 * (kHeadDim / 4); x += 256)
-      reinterpret_cast<float4*>(zs)[x] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int t = 0; t < kZRows * kZChunk / 256; ++t) {
-      const int x = tid + 256 * t;
-      const int r = x / kZChunk, jj = x % kZChunk;
-      ms[x] = (r < rows && jj < jn) ? __bfloat162float(mh[static_cast<size_t>(r) * nBp + j0 + jj]) : 0.f;
-    }
-    cp_async_wait<0>();
-    __syncthreads();
-    const float* mrow = ms + g * (kZRows / 2) * kZChunk;
-    for (int jj = 0; jj < jn4; jj += 4) {
-      const float z0 = zs[(jj + 0) * kHeadDim + c], z1 = zs[(jj + 1) * kHeadDim + c];
-      const float z2 = zs[(jj + 2) * kHeadDim + c], z3 = zs[(jj + 3) * kHeadDim + c];
-#pragma unroll
-      for (int r = 0; r < kZRows / 2; ++r) {
-        const float4 mv = *reinterpret_cast<const float4*>(mrow + r * kZChunk + jj);
-        acc[r] = fmaf(mv.x, z0, acc[r]);
-        acc[r] = fmaf(mv.y, z1, acc[r]);
-        acc[r] = fmaf(mv.z, z2, acc[r]);
-        acc[r] = fmaf(mv.w, z3, acc[r]);
-      }
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < kZRows / 2; ++r) {
-    const int row = g * (kZRows / 2) + r;
-    if (row < rows) Z[(static_cast<size_t>(bh) * nB + i0 + row) * kHeadDim + c] = acc[r];
+// ------------------------------------------------------------------ z -> bf16
+// z_j rounded to bf16 (RNE): the B operand of the Z column tile of hgemm_kernel.
+__global__ void __launch_bounds__(256) zb_kernel(const float4* __restrict__ z,
+                                                 uint2* __restrict__ zb, size_t n4) {
+  for (size_t x = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; x < n4;
+       x += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 v = z[x];
+    zb[x] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
   }
 }
 
@@ -333,11 +353,13 @@ cudaError_t launch_linear(const Dims& g, const void* q, float sm_scale, const vo
   __nv_bfloat16* Hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.Hbuf);
   float* Zbuf = reinterpret_cast<float*>(ws + L.Zbuf);
   __nv_bfloat16* Ol = reinterpret_cast<__nv_bfloat16*>(ws + L.Ol);
+  __nv_bfloat16* Zb = reinterpret_cast<__nv_bfloat16*>(ws + L.Zb);
 
-  CUtensorMap tmA, tmB, tmH;
+  CUtensorMap tmA, tmB, tmZ, tmH;
   if (!make_tmap_3d(&tmA, mask, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.nBp, g.nB, g.BH, 64, 128) ||
       !make_tmap_3d(&tmB, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim * kHeadDim, g.nB, g.BH, 64,
                     64) ||
+      !make_tmap_3d(&tmZ, Zb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim, g.nB, g.BH, 64, 64) ||
       !make_tmap_3d(&tmH, Hbuf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim,
                     static_cast<uint64_t>(g.nB) * kHeadDim, g.BH, 64, 128))
     return cudaErrorInvalidValue;
@@ -346,18 +368,23 @@ cudaError_t launch_linear(const Dims& g, const void* q, float sm_scale, const vo
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(linout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(zsum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kZSmem);
-  if (e != cudaSuccess) return e;
 
   {
-    TraceScope ts_("hgemm_kernel", st);
-    hgemm_kernel<<<dim3(kHeadDim * kHeadDim / 128, (g.nB + 127) / 128, g.BH), 128, kGemmSmem, st>>>(
-      tmA, tmB, Hbuf, g.nB, status);
+    TraceScope ts_("zb_kernel", st);
+    const size_t n4 = static_cast<size_t>(g.BH) * g.nB * kHeadDim / 4;
+    const int blocks = static_cast<int>((n4 + 255) / 256 < 4096 ? (n4 + 255) / 256 : 4096);
+    zb_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(z), reinterpret_cast<uint2*>(Zb), n4);
   }
   {
-    TraceScope ts_("zsum_kernel", st);
-    zsum_kernel<<<dim3((g.nB + kZRows - 1) / kZRows, g.BH), 256, kZSmem, st>>>(
-      z, static_cast<const __nv_bfloat16*>(mask), Zbuf, g.nB, g.nBp);
+    TraceScope ts_("hgemm_kernel", st);
+    const int n_mt = (g.nB + 127) / 128;
+    const int n_tiles = (kHeadDim * kHeadDim / 128 + 1) * n_mt * g.BH;
+    int dev = 0, n_sm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = n_tiles < 2 * n_sm ? n_tiles : 2 * n_sm;
+    hgemm_kernel<<<grid, kGemmThreads, kGemmSmem, st>>>(tmA, tmB, tmZ, Hbuf, Zbuf, g.nB, n_mt, n_tiles,
+                                                         status);
   }
   {
     TraceScope ts_("linout_kernel", st);

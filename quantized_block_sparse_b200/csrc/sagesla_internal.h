@@ -26,6 +26,7 @@ struct WsLayout {
   size_t mu_part;    // fp32 [BH, nB, d]   per-block channel sums of K
   size_t Hbuf;       // bf16 [BH, nB, d, d]
   size_t Zbuf;       // fp32 [BH, nB, d]
+  size_t Zb;         // bf16 [BH, nB, d]      z rounded to bf16 (the Z GEMM operand)
   size_t Ol;         // bf16 [BH, N, d]
   size_t total;
 };
