@@ -28,6 +28,10 @@ WsLayout ws_layout(const Dims& g) {
   off = align256(off + static_cast<size_t>(g.BH) * g.nB * kHeadDim * 4);
   L.Zb = off;
   off = align256(off + static_cast<size_t>(g.BH) * g.nB * kHeadDim * 2);
+  L.pairs = off;
+  off = align256(off + static_cast<size_t>(g.BH) * g.nB * 8);
+  L.pair_counts = off;
+  off = align256(off + static_cast<size_t>(g.BH) * ((g.nB + 63) / 64) * 4);
   L.Ol = off;
   off = align256(off + static_cast<size_t>(g.BH) * g.N * kHeadDim * 2);
   L.total = off;

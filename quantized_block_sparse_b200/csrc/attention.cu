@@ -29,6 +29,9 @@
 namespace sgs {
 namespace {
 
+constexpr int kPairWindow = 32;   // pairing: candidates per query block
+constexpr int kPairSegment = 64;  // pairing: query blocks per segment (one CTA)
+
 // K tiles (8 KB, read only by QK^T) and V tiles (16 KB, read by P.V after the softmax) sit
 // in separate rings: a K slot frees as soon as its QK^T completes, so K runs far ahead;
 // a V slot frees when its P.V completes.
@@ -64,7 +67,8 @@ constexpr int kPolyReps = 0;
 // release/acquire).
 struct StageMeta {
   int j;       // key block
-  int flags;   // bit 0: critical for query block i0, bit 1: for i0+1, bit 2: last step
+  int flags;   // bit 0: critical for the pair's first query block, bit 1: for the second,
+               // bit 2: last step
   float sk;    // k_scale of block j
   int pad;
 };
@@ -75,13 +79,15 @@ constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColO = 128;
 
 struct AttnParams {
+  const int2* pairs;       // [BH][nB]: (first, second) query block of each tile; -1 = none
+  const int* pair_counts;  // [BH][n_seg]: tiles per segment of 64 query blocks
   const float* q_scale;
   const float* k_scale;
   const int32_t* crit;
   const __nv_bfloat16* Ol;  // nullptr when there is no marginal block
   __nv_bfloat16* out;
   int* status;
-  int N, nB, k_c;
+  int N, nB, k_c, n_seg;
 };
 
 struct UnionWalk {
@@ -124,11 +130,6 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
 __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
 
@@ -256,19 +257,7 @@ __device__ __forceinline__ float quad_sum(float v) {
   return v + __shfl_xor_sync(0xffffffffu, v, 2);
 }
 
-__device__ __forceinline__ void tmem_st32_sync(uint32_t taddr, const uint32_t (&r)[32]) {
-  tmem_st32(taddr, r);
-  tmem_wait_st();
-}
 
-// tcgen05.mma kind::f16 with the A operand (P, M x K) read from TMEM.
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
-}
 
 // Same, with the disable-output-lane mask: bit k of the 128-bit mask (m0 = lanes 0-31, ...,
 // m3 = lanes 96-127) keeps D lane k unchanged. Used for union steps that are critical for
@@ -311,14 +300,21 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 
   const int pr = blockIdx.x, bh = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int i0 = 2 * pr;
   const int nB = p.nB;
+  int tile = pr, seg = 0;  // tile pr of the head: entry tile of segment seg
+  {
+    const int* cnt = p.pair_counts + static_cast<size_t>(bh) * p.n_seg;
+    while (seg < p.n_seg && tile >= __ldg(cnt + seg)) tile -= __ldg(cnt + seg++);
+  }
+  if (seg >= p.n_seg) return;  // past the head's last tile (whole CTA, before any barrier)
+  const int2 pq = p.pairs[static_cast<size_t>(bh) * nB + seg * kPairSegment + tile];
+  const int i0 = pq.x, i1 = pq.y;  // rows 0-63: block i0; rows 64-127: block i1 (-1: none)
 
   UnionWalk walk;
   walk.c0 = p.crit + (static_cast<size_t>(bh) * nB + i0) * p.k_c;
-  walk.c1 = walk.c0 + p.k_c;
+  walk.c1 = p.crit + (static_cast<size_t>(bh) * nB + (i1 >= 0 ? i1 : i0)) * p.k_c;
   walk.n0 = p.k_c;
-  walk.n1 = (i0 + 1 < nB) ? p.k_c : 0;
+  walk.n1 = (i1 >= 0) ? p.k_c : 0;
   walk.p0 = 0;
   walk.p1 = 0;
 
@@ -362,7 +358,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     if (lane == 0) {
       mbar_expect_tx(smem_u32(q_full), 16384);
       tma_load_3d(sQ, &tmQ, smem_u32(q_full), 0, i0 * 64, bh);
-      tma_load_3d(sQ + 8192, &tmQ, smem_u32(q_full), 0, i0 * 64 + 64, bh);
+      tma_load_3d(sQ + 8192, &tmQ, smem_u32(q_full), 0, (i1 >= 0 ? i1 : i0) * 64, bh);
       int j, fl;
       bool have = walk.next(j, fl);  // k_c >= 1: at least one step
       int tK = 0, tV = 0, nsteps = -1;  // nsteps: known once the walk is exhausted
@@ -516,7 +512,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     // Warp w owns the 16 TMEM lanes LB = 32*(w%4) + 16*((w-2)/4) .. LB+15 (query rows of the
     // 128-row tile); in the 16-lane load shape thread t holds rows LB + t/4 and LB + t/4 + 8,
     // 16 keys each, and the four threads of a quad (t/4) share rows. Rows 0-63 are block i0,
-    // 64-127 block i0+1, so membership is warp-uniform. A warp whose half is not critical
+    // 64-127 block i1, so membership is warp-uniform. A warp whose half is not critical
     // for a step skips it (the P.V MMA masks its rows).
     const int wq = warp & 3;
     const int sub = (warp - 2) >> 2;
@@ -524,8 +520,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const int q = lane & 3;
     const int rr0 = static_cast<int>(lb) + (lane >> 2);  // rows rr0 and rr0 + 8
     const int half = rr0 >> 6;
-    const int i = i0 + half;
-    const float sq = (i < nB) ? p.q_scale[static_cast<size_t>(bh) * nB + i] : 0.f;
+    const int i = half ? i1 : i0;
+    const float sq = (i >= 0) ? p.q_scale[static_cast<size_t>(bh) * nB + i] : 0.f;
     const uint32_t lane_off = lb << 16;
     {  // O starts at zero for these rows; every P.V then accumulates
       uint32_t z[32];
@@ -668,9 +664,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     // Epilogue layout: warp w reads its quadrant's 32 lanes (32x32b), one row per thread,
     // output columns [64*sub, 64*sub + 64).
     const int r = 32 * wq + lane;
-    const int ie = i0 + (r >> 6);
+    const int ie = (r >> 6) ? i1 : i0;
     const int tok = ie * 64 + (r & 63);
-    const bool row_valid = (ie < nB) && (tok < p.N);
+    const bool row_valid = (ie >= 0) && (tok < p.N);
     const uint32_t eoff = static_cast<uint32_t>(32 * wq) << 16;
     if (ok) {
       const float inv = 1.f / rowsum[r];
@@ -717,6 +713,69 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   if (warp == 1) tmem_dealloc(taddr, kTmemCols);
 }
 
+// Pairs of query blocks for the attention tiles. Two blocks that share many critical key
+// blocks make a short union walk: the tile executes |crit(i0) U crit(i1)| steps for 2*k_c
+// useful ones. One CTA per (head, segment of 64 query blocks): the segment's blocks are
+// taken in ascending order and each unpaired block is matched with the unpaired block
+// among the next 32 of the segment that shares the most critical blocks (ties: the
+// nearest), or left alone. Segment s writes its n_s tiles, (i0, i1) with i1 = -1 for a
+// block left alone, to pairs[bh][64*s + k] and n_s to counts[bh][s]; tile t of a head is
+// then entry t - (n_0 + ... + n_{s-1}) of the segment s where that sum passes t.
+__global__ void __launch_bounds__(256) pair_kernel(const int32_t* __restrict__ crit, int nB, int k_c,
+                                                   int2* __restrict__ pairs, int* __restrict__ counts) {
+  extern __shared__ uint32_t psm[];
+  const int seg = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  const int lo = seg * kPairSegment, hi = min(nB, lo + kPairSegment), rows = hi - lo;
+  const int nW = ((nB + 31) >> 5) | 1;  // words per membership row, odd: no bank conflicts
+  uint32_t* bits = psm;                                                                // [rows][nW]
+  uint8_t* ov = reinterpret_cast<uint8_t*>(bits + static_cast<size_t>(kPairSegment) * nW);  // [rows][32]
+  for (int x = tid; x < rows * nW; x += 256) bits[x] = 0u;
+  __syncthreads();
+  const int32_t* cb = crit + (static_cast<size_t>(bh) * nB + lo) * k_c;
+  const int total = rows * k_c;
+  for (int x0 = tid; x0 < total; x0 += 256 * 16) {  // 16 loads in flight per thread
+    int jv[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) jv[u] = (x0 + 256 * u < total) ? __ldg(cb + x0 + 256 * u) : -1;
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      if (jv[u] >= 0) atomicOr(&bits[((x0 + 256 * u) / k_c) * nW + (jv[u] >> 5)], 1u << (jv[u] & 31));
+  }
+  __syncthreads();
+  // ov[r][d-1] = |crit(lo+r) ^ crit(lo+r+d)| for d = 1..32 inside the segment (0 past it)
+  for (int x = tid; x < rows * kPairWindow; x += 256) {
+    const int r = x / kPairWindow, r2 = r + 1 + x % kPairWindow;
+    int v = 0;
+    if (r2 < rows)
+      for (int w = 0; w < nW; ++w) v += __popc(bits[r * nW + w] & bits[r2 * nW + w]);
+    ov[x] = static_cast<uint8_t>(min(v, 254));
+  }
+  __syncthreads();
+  if (tid < 32) {
+    int2* out = pairs + static_cast<size_t>(bh) * nB + lo;
+    unsigned long long used = 0ull;  // bit k: row r + k already in a tile (warp-uniform)
+    int np = 0;
+    unsigned nxt = ov[lane];
+    for (int r = 0; r < rows; ++r) {
+      const unsigned cur = nxt;
+      if (r + 1 < rows) nxt = ov[(r + 1) * kPairWindow + lane];
+      if (used & 1ull) {
+        used >>= 1;
+        continue;
+      }
+      const bool ok = r + 1 + lane < rows && !((used >> (1 + lane)) & 1ull);
+      const unsigned key = ok ? ((cur + 1u) << 5) | (31u - static_cast<unsigned>(lane)) : 0u;
+      const unsigned best = __reduce_max_sync(0xffffffffu, key);
+      const int d = best ? 1 + (31 - static_cast<int>(best & 31u)) : 0;
+      if (lane == 0) out[np] = make_int2(lo + r, d ? lo + r + d : -1);
+      ++np;
+      if (d) used |= 1ull << d;
+      used >>= 1;
+    }
+    if (lane == 0) counts[static_cast<size_t>(bh) * gridDim.x + seg] = np;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_attention(const Dims& g, const int8_t* q8, const int8_t* k8,
@@ -731,7 +790,21 @@ cudaError_t launch_attention(const Dims& g, const int8_t* q8, const int8_t* k8,
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
   if (e != cudaSuccess) return e;
+  int2* pairs = reinterpret_cast<int2*>(ws + L.pairs);
+  int* pair_counts = reinterpret_cast<int*>(ws + L.pair_counts);
+  const int n_seg = (g.nB + kPairSegment - 1) / kPairSegment;
+  {
+    const int nW = ((g.nB + 31) >> 5) | 1;
+    const int psmem = kPairSegment * nW * 4 + kPairSegment * kPairWindow;
+    e = cudaFuncSetAttribute(pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, psmem);
+    if (e != cudaSuccess) return e;
+    TraceScope ts_("pair_kernel", st);
+    pair_kernel<<<dim3(n_seg, g.BH), 256, psmem, st>>>(crit, g.nB, k_c, pairs, pair_counts);
+  }
   AttnParams p;
+  p.pairs = pairs;
+  p.pair_counts = pair_counts;
+  p.n_seg = n_seg;
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.crit = crit;
@@ -743,7 +816,7 @@ cudaError_t launch_attention(const Dims& g, const int8_t* q8, const int8_t* k8,
   p.k_c = k_c;
   {
     TraceScope ts_("attn_kernel", st);
-    attn_kernel<<<dim3((g.nB + 1) / 2, g.BH), kAttnThreads, kAttnSmem, st>>>(tmQ, tmK, tmV, p);
+    attn_kernel<<<dim3(g.nB, g.BH), kAttnThreads, kAttnSmem, st>>>(tmQ, tmK, tmV, p);
   }
   return cudaGetLastError();
 }

@@ -27,6 +27,8 @@ struct WsLayout {
   size_t Hbuf;       // bf16 [BH, nB, d, d]
   size_t Zbuf;       // fp32 [BH, nB, d]
   size_t Zb;         // bf16 [BH, nB, d]      z rounded to bf16 (the Z GEMM operand)
+  size_t pairs;      // int2 [BH, nB]         query-block pairs of the attention tiles
+  size_t pair_counts;  // int32 [BH, ceil(nB/64)] tiles per pairing segment
   size_t Ol;         // bf16 [BH, N, d]
   size_t total;
 };
