@@ -141,6 +141,7 @@ __device__ __forceinline__ float phi_f32(float x) { return x > 0.f ? __fadd_rn(x
 // bulk copies for the raw Q and K rows, two TMA boxes for V straight into the MN-major
 // 128-byte-swizzled operand tile), so a CTA keeps 48 KB in flight and three CTAs share an SM.
 __global__ void __launch_bounds__(kPrepThreads, 3) prep_block_kernel(const __grid_constant__ CUtensorMap tmV,
+                                                                   const __grid_constant__ CUtensorMap tmH,
                                                                    PrepParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -281,24 +282,33 @@ __global__ void __launch_bounds__(kPrepThreads, 3) prep_block_kernel(const __gri
   if (!mbar_wait(smem_u32(bar + 1), 0, &abort_flag, p.status)) mbar_wait_inflight(smem_u32(bar + 1), 0, p.status);
   tc_fence_after();
 
-  // h_j[c][e]: TMEM lane c, column e. Warps w and w+4 split the 128 columns.
+  // h_j[c][e]: TMEM lane c, column e. Warps w and w+4 split the 128 columns. The bf16 rows
+  // are staged over the raw Q/K rows (dead by now) as two 128-row x 64-column tiles in the
+  // 128-byte-swizzled layout (conflict-free 16-byte writes) and leave by two TMA stores.
+  unsigned char* sH = smem + 32768;
   if (!abort_flag) {
     const int cl = 32 * (warp & 3) + lane;
-    const int col0 = 64 * (warp >> 2);
+    const int half = warp >> 2;
     uint32_t rr[64];
-    tmem_ld64_sync(taddr + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + col0, rr);
-    uint4* dst = reinterpret_cast<uint4*>(p.h + (blk * kHeadDim + cl) * kHeadDim + col0);
+    tmem_ld64_sync(taddr + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + 64 * half, rr);
+    const uint32_t tile = smem_u32(sH) + half * 16384;
 #pragma unroll
     for (int q = 0; q < 8; ++q)
-      dst[q] = make_uint4(pack_bf16x2(__uint_as_float(rr[8 * q]), __uint_as_float(rr[8 * q + 1])),
-                          pack_bf16x2(__uint_as_float(rr[8 * q + 2]), __uint_as_float(rr[8 * q + 3])),
-                          pack_bf16x2(__uint_as_float(rr[8 * q + 4]), __uint_as_float(rr[8 * q + 5])),
-                          pack_bf16x2(__uint_as_float(rr[8 * q + 6]), __uint_as_float(rr[8 * q + 7])));
+      st_shared_v4(tile + sw128_offset(cl, q), pack_bf16x2(__uint_as_float(rr[8 * q]), __uint_as_float(rr[8 * q + 1])),
+                   pack_bf16x2(__uint_as_float(rr[8 * q + 2]), __uint_as_float(rr[8 * q + 3])),
+                   pack_bf16x2(__uint_as_float(rr[8 * q + 4]), __uint_as_float(rr[8 * q + 5])),
+                   pack_bf16x2(__uint_as_float(rr[8 * q + 6]), __uint_as_float(rr[8 * q + 7])));
+    fence_async_smem();
   }
   if (tid >= 128) p.z[blk * kHeadDim + c] = zacc;
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(taddr, 128);
+  if (tid == 0 && !abort_flag) {
+    tma_store_3d(&tmH, smem_u32(sH), 0, j * kHeadDim, bh);
+    tma_store_3d(&tmH, smem_u32(sH) + 16384, 64, j * kHeadDim, bh);
+    bulk_store_commit_wait_read();
+  }
 }
 
 }  // namespace
@@ -319,8 +329,10 @@ cudaError_t launch_prepare(const Dims& g, const void* q, const void* k, const vo
     TraceScope ts_("kmean_kernel", st);
     kmean_kernel<<<dim3(g.BH, kHeadDim / 16), 256, 0, st>>>(part, k_mean, g.N, g.nB);
   }
-  CUtensorMap tmV;
-  if (!make_tmap_3d(&tmV, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim, g.N, g.BH, 64, 64))
+  CUtensorMap tmV, tmH;
+  if (!make_tmap_3d(&tmV, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim, g.N, g.BH, 64, 64) ||
+      !make_tmap_3d(&tmH, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim,
+                    static_cast<uint64_t>(g.nB) * kHeadDim, g.BH, 64, 128))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(prep_block_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem);
@@ -345,7 +357,7 @@ cudaError_t launch_prepare(const Dims& g, const void* q, const void* k, const vo
   p.Npad = g.Npad;
   {
     TraceScope ts_("prep_block_kernel", st);
-    prep_block_kernel<<<dim3(g.nB, g.BH), kPrepThreads, kPrepSmem, st>>>(tmV, p);
+    prep_block_kernel<<<dim3(g.nB, g.BH), kPrepThreads, kPrepSmem, st>>>(tmV, tmH, p);
   }
   return cudaGetLastError();
 }
