@@ -23,14 +23,15 @@ namespace sgs {
 namespace {
 
 // ------------------------------------------------------------------ H = M . h
-// Persistent tcgen05 GEMM: each CTA walks output tiles (128 query blocks x 128 columns of
-// h's d*d, N fastest so consecutive tiles share the mask tile in L2). Warp 0 streams A/B
-// k-blocks through a 3-stage ring with TMA, warp 1 issues the MMAs into one of two TMEM
-// accumulators, warps 2-5 drain the other accumulator (bf16) while the next tile runs.
-// One more column tile per row block computes Z = M . z from z rounded to bf16 (the same
-// operand precision as h) and is written in fp32.
-constexpr int kGemmStages = 3;
-constexpr int kGemmStageBytes = 16384 + 16384;
+// Persistent tcgen05 GEMM, one CTA per SM: each CTA walks output tiles (128 query blocks x
+// 256 columns of h's d*d, N fastest so consecutive tiles share the mask tile in L2; 256-wide
+// tiles halve the mask re-reads, the main L2 traffic). Warp 0 streams A/B k-blocks through
+// a 4-stage ring with TMA, warp 1 issues the MMAs (M128 N256 K16) into one of two 256-column
+// TMEM accumulators, warps 2-5 drain the other accumulator (bf16) while the next tile runs.
+// One more, 128-column tile per row block computes Z = M . z from z rounded to bf16 (the
+// same operand precision as h) and is written in fp32.
+constexpr int kGemmStages = 4;
+constexpr int kGemmStageBytes = 16384 + 32768;
 constexpr int kGemmThreads = 192;
 constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + 1024 + 256;
 
@@ -51,7 +52,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_con
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   __shared__ int abort_flag;
 
-  constexpr int kNTH = kHeadDim * kHeadDim / 128;  // 128 N-tiles of H
+  constexpr int kNTH = kHeadDim * kHeadDim / 256;  // 64 N-tiles of H
   constexpr int kNT = kNTH + 1;                     // + the Z tile
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nK = (nB + 63) / 64;
@@ -71,7 +72,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_con
     prefetch_tmap(&tmB);
     prefetch_tmap(&tmZ);
   }
-  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 256);
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -92,11 +93,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_con
           }
           const uint32_t sa = smem_u32(smem + s * kGemmStageBytes);
           const uint32_t sb = sa + 16384;
-          mbar_expect_tx(smem_u32(full + s), kGemmStageBytes);
+          mbar_expect_tx(smem_u32(full + s), nt < kNTH ? kGemmStageBytes : 16384 + 16384);
           tma_load_3d(sa, &tmA, smem_u32(full + s), kb * 64, mt * 128, bh);
           if (nt < kNTH) {
-            tma_load_3d(sb, &tmB, smem_u32(full + s), nt * 128, kb * 64, bh);
-            tma_load_3d(sb + 8192, &tmB, smem_u32(full + s), nt * 128 + 64, kb * 64, bh);
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+              tma_load_3d(sb + 8192 * g, &tmB, smem_u32(full + s), nt * 256 + 64 * g, kb * 64, bh);
           } else {
             tma_load_3d(sb, &tmZ, smem_u32(full + s), 0, kb * 64, bh);
             tma_load_3d(sb + 8192, &tmZ, smem_u32(full + s), 64, kb * 64, bh);
@@ -109,7 +111,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_con
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc(1, 1, 0, 1, 128, 128);
+      constexpr uint32_t idesc_h = make_idesc(1, 1, 0, 1, 128, 256);
+      constexpr uint32_t idesc_z = make_idesc(1, 1, 0, 1, 128, 128);
       int it = 0, lt = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++lt) {
@@ -119,6 +122,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_con
           break;
         }
         tc_fence_after();
+        const uint32_t idesc = (tile % kNT) < kNTH ? idesc_h : idesc_z;
         for (int kb = 0; kb < nK; ++kb, ++it) {
           const int s = it % kGemmStages;
           if (!mbar_wait(smem_u32(full + s), (it / kGemmStages) & 1, &abort_flag, status)) {
@@ -130,7 +134,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_con
           const uint32_t sb = sa + 16384;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(taddr + 128 * a, make_sdesc(sa + kk * 32, 16, 1024),
+            mma_bf16(taddr + 256 * a, make_sdesc(sa + kk * 32, 16, 1024),
                      make_sdesc(sb + kk * 2048, 8192, 1024), idesc, (kb | kk) != 0);
           mma_commit(smem_u32(empty + s));
         }
@@ -151,11 +155,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_con
       tc_fence_after();
       const int i = mt * 128 + 32 * wq + lane;
       if (nt < kNTH) {
-        __nv_bfloat16* dst = Hout + (static_cast<size_t>(bh) * nB + i) * (kHeadDim * kHeadDim) + nt * 128;
+        __nv_bfloat16* dst = Hout + (static_cast<size_t>(bh) * nB + i) * (kHeadDim * kHeadDim) + nt * 256;
 #pragma unroll
-        for (int cchunk = 0; cchunk < 4; ++cchunk) {
+        for (int cchunk = 0; cchunk < 8; ++cchunk) {
           uint32_t r[32];
-          tmem_ld32_sync(taddr + (static_cast<uint32_t>(32 * wq) << 16) + 128 * a + 32 * cchunk, r);
+          tmem_ld32_sync(taddr + (static_cast<uint32_t>(32 * wq) << 16) + 256 * a + 32 * cchunk, r);
           if (i < nB) {
             uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cchunk);
 #pragma unroll
@@ -171,7 +175,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_con
 #pragma unroll
         for (int cchunk = 0; cchunk < 4; ++cchunk) {
           uint32_t r[32];
-          tmem_ld32_sync(taddr + (static_cast<uint32_t>(32 * wq) << 16) + 128 * a + 32 * cchunk, r);
+          tmem_ld32_sync(taddr + (static_cast<uint32_t>(32 * wq) << 16) + 256 * a + 32 * cchunk, r);
           if (i < nB) {
             uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cchunk);
 #pragma unroll
@@ -185,7 +189,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_con
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(taddr, 256);
+  if (warp == 1) tmem_dealloc(taddr, 512);
 }
 
 // ------------------------------------------------------------------ z -> bf16
@@ -207,7 +211,7 @@ __global__ void __launch_bounds__(256) zb_kernel(const float4* __restrict__ z,
 // two 128x128 products back (a quadrant of rows and half of the columns each), scale by
 // 1/den and stage O_l over the H tiles (swizzled) for four TMA stores.
 constexpr int kLinThreads = 256;
-constexpr int kLinSmem = 32768 + 65536 + 1024 + 1024 + 256;
+constexpr int kLinSmem = 32768 + 65536 + 1024 + 1024 + 1024 + 256;
 
 __global__ void __launch_bounds__(kLinThreads) linout_kernel(const __grid_constant__ CUtensorMap tmH,
                                                              const __grid_constant__ CUtensorMap tmQ,
@@ -219,8 +223,9 @@ __global__ void __launch_bounds__(kLinThreads) linout_kernel(const __grid_consta
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   unsigned char* sA = smem;            // Q, then phi(Q~): 2 column blocks x 128 rows x 128 B
   unsigned char* sH = smem + 32768;    // H_i0, H_i1: each 2 e-groups x 128 c rows x 128 B
-  float* dpart = reinterpret_cast<float*>(smem + 32768 + 65536);  // [2][128] denominator halves
-  uint64_t* lfull = reinterpret_cast<uint64_t*>(smem + 32768 + 65536 + 1024);  // Q and H landed
+  float* dpart = reinterpret_cast<float*>(smem + 32768 + 65536);         // [2][128] denominator halves
+  float* sZ = reinterpret_cast<float*>(smem + 32768 + 65536 + 1024);     // Z_i0, Z_i1 [2][128]
+  uint64_t* lfull = reinterpret_cast<uint64_t*>(smem + 32768 + 65536 + 2048);  // Q, H, Z landed
   uint64_t* mdone = lfull + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + 1);
   __shared__ int abort_flag;
@@ -233,7 +238,10 @@ __global__ void __launch_bounds__(kLinThreads) linout_kernel(const __grid_consta
     mbar_init(smem_u32(lfull), 1);
     mbar_init(smem_u32(mdone), 1);
     fence_mbar_init();
-    mbar_expect_tx(smem_u32(lfull), (two ? 65536 : 32768) + 32768);
+    mbar_expect_tx(smem_u32(lfull), (two ? 65536 + 1024 : 32768 + 512) + 32768);
+    for (int b = 0; b < (two ? 2 : 1); ++b)
+      bulk_load(smem_u32(sZ) + b * 512, Z + (static_cast<size_t>(bh) * nB + i0 + b) * kHeadDim, 512,
+                smem_u32(lfull));
     for (int b = 0; b < (two ? 2 : 1); ++b) {
       const uint32_t dst = smem_u32(sH) + b * 32768;
       tma_load_3d(dst, &tmH, smem_u32(lfull), 0, (i0 + b) * 128, bh);
@@ -258,7 +266,7 @@ __global__ void __launch_bounds__(kLinThreads) linout_kernel(const __grid_consta
   {
     const int r = tid & 127, chh = tid >> 7;
     const int i = i0 + (r >> 6);
-    const float* zr = Z + (static_cast<size_t>(bh) * nB + (i < nB ? i : 0)) * kHeadDim + 64 * chh;
+    const float* zr = sZ + ((i < nB) ? (r >> 6) : 0) * kHeadDim + 64 * chh;
     const uint32_t tile = smem_u32(sA) + chh * 16384;
     float dacc = 0.f;
 #pragma unroll
@@ -380,11 +388,11 @@ cudaError_t launch_linear(const Dims& g, const void* q, float sm_scale, const vo
   {
     TraceScope ts_("hgemm_kernel", st);
     const int n_mt = (g.nB + 127) / 128;
-    const int n_tiles = (kHeadDim * kHeadDim / 128 + 1) * n_mt * g.BH;
+    const int n_tiles = (kHeadDim * kHeadDim / 256 + 1) * n_mt * g.BH;
     int dev = 0, n_sm = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-    const int grid = n_tiles < 2 * n_sm ? n_tiles : 2 * n_sm;
+    const int grid = n_tiles < n_sm ? n_tiles : n_sm;
     hgemm_kernel<<<grid, kGemmThreads, kGemmSmem, st>>>(tmA, tmB, tmZ, Hbuf, Zbuf, g.nB, n_mt, n_tiles,
                                                          status);
   }
