@@ -240,11 +240,14 @@ class SageSLA:
         self.sel = alloc_selection(B, H, N, rho, nu, device, logits)
         self.out = torch.empty(B, H, N, HEAD_DIM, dtype=torch.bfloat16, device=device)
 
-    def __call__(self, q, k, v, stream=None):
+    def __call__(self, q, k, v, stream=None, out=None):
+        """One SageSLA call; the result goes to `out` (bf16 [B,H,N,128]) or the engine's own
+        output buffer."""
         sagesla_prepare(q, k, v, self.workspace, out=self.prep, stream=stream)
         sagesla_select(self.prep.q_bar, self.prep.k_bar, self.N, self.rho, self.nu, out=self.sel,
                        stream=stream)
-        return sagesla_forward(q, v, self.prep, self.sel, self.workspace, out=self.out, stream=stream)
+        return sagesla_forward(q, v, self.prep, self.sel, self.workspace,
+                               out=self.out if out is None else out, stream=stream)
 
     def check(self, stream=None):
         sagesla_check_status(self.workspace, stream)
