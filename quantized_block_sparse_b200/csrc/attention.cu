@@ -204,17 +204,26 @@ __device__ __forceinline__ void tmem_st_16x128b_x8(uint32_t taddr, const uint32_
 // mantissa). P = 2^((A - 1.5*2^23)*sc - m_row), rounded to bf16 pairs in pk (16x128b order);
 // returns the fp32 sums of this thread's P per row. Keys >= nvalid (a ragged last key block)
 // get P = 0.
-template <bool RAGGED>
+// FOLD: x = A*sc + (-m - 1.5*2^23*sc) in one FMA instead of (A - 1.5*2^23)*sc - m. The
+// product is exact inside the FMA, so the only extra error is the rounding of the constant,
+// at most half an ulp of 1.5*2^23*sc + m; callers fold only when 1.5*2^23*sc < 2^14, which
+// bounds it by 2^-10 (log2 units; P within 0.07 %, below its own bf16 rounding). The error
+// is common to a row's keys of one tile.
+constexpr float kFoldLimit = 16384.f;
+template <bool RAGGED, bool FOLD>
 __device__ __forceinline__ void softmax_tile(const float (&A)[32], float sc, float negm0,
                                              float negm1, int q, int nvalid, uint32_t (&pk)[16],
                                              float& ps0, float& ps1) {
   const uint64_t sub = f2pack(-kMagic, -kMagic), sc2 = f2pack(sc, sc);
-  const uint64_t nm0 = f2pack(negm0, negm0), nm1 = f2pack(negm1, negm1);
+  const float msc = __fmul_rn(kMagic, sc);
+  const float c0 = FOLD ? __fsub_rn(negm0, msc) : negm0, c1 = FOLD ? __fsub_rn(negm1, msc) : negm1;
+  const uint64_t nm0 = f2pack(c0, c0), nm1 = f2pack(c1, c1);
   uint64_t acc0 = 0ull, acc1 = 0ull;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    const uint64_t x0 = fma2(add2(f2pack(A[4 * k], A[4 * k + 1]), sub), sc2, nm0);
-    const uint64_t x1 = fma2(add2(f2pack(A[4 * k + 2], A[4 * k + 3]), sub), sc2, nm1);
+    const uint64_t a01 = f2pack(A[4 * k], A[4 * k + 1]), a23 = f2pack(A[4 * k + 2], A[4 * k + 3]);
+    const uint64_t x0 = fma2(FOLD ? a01 : add2(a01, sub), sc2, nm0);
+    const uint64_t x1 = fma2(FOLD ? a23 : add2(a23, sub), sc2, nm1);
     float a0, a1, b0, b1, pa0, pa1, pb0, pb1;
     f2unpack(x0, a0, a1);
     f2unpack(x1, b0, b1);
@@ -565,10 +574,17 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         const float sc = __fmul_rn(__fmul_rn(sq, skj), kLog2e);
         uint32_t pk[16];
         float ps0, ps1;
-        if (ragged)
-          softmax_tile<true>(A, sc, -m0, -m1, q, nvalid, pk, ps0, ps1);
-        else
-          softmax_tile<false>(A, sc, -m0, -m1, q, 64, pk, ps0, ps1);
+        const bool fold = __fmul_rn(kMagic, sc) < kFoldLimit;  // warp-uniform
+        auto run_tile = [&]() {
+          if (ragged) {
+            if (fold) softmax_tile<true, true>(A, sc, -m0, -m1, q, nvalid, pk, ps0, ps1);
+            else softmax_tile<true, false>(A, sc, -m0, -m1, q, nvalid, pk, ps0, ps1);
+          } else {
+            if (fold) softmax_tile<false, true>(A, sc, -m0, -m1, q, 64, pk, ps0, ps1);
+            else softmax_tile<false, false>(A, sc, -m0, -m1, q, 64, pk, ps0, ps1);
+          }
+        };
+        run_tile();
         // rare path: raise m where a partial sum left [0, 2^24] (quad-consistent decision)
         bool need0 = !(ps0 <= kPsumLimit), need1 = !(ps1 <= kPsumLimit);
         need0 = quad_any(need0);
@@ -604,10 +620,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             if (m1 != -INFINITY) alpha1 = ex2_approx(m1 - mt);
             m1 = mt;
           }
-          if (ragged)
-            softmax_tile<true>(A, sc, -m0, -m1, q, nvalid, pk, ps0, ps1);
-          else
-            softmax_tile<false>(A, sc, -m0, -m1, q, 64, pk, ps0, ps1);
+          run_tile();
         }
         l0 = fmaf(l0, alpha0, ps0);
         l1 = fmaf(l1, alpha1, ps1);
