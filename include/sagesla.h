@@ -128,9 +128,12 @@ int sagesla_select(const sagesla_shape* shape, const float* q_bar, const float* 
 /* Steps (5)-(7).
  * Inputs : q bf16 [B,H,N,d] (phi(Q~) is recomputed from it), sm_scale, and the
  *          outputs of prepare and select; k_c and m must be the counts of select.
- *          v bf16 [B,H,N,d].
+ *          v bf16 [B,H,N,d]. The marginal sums H_i = sum h_j and Z_i = sum z_j are
+ *          computed as one GEMM with marg_mask; marg_idx (the same set as a list) is
+ *          checked for alignment but not read (it may be NULL when m == 0).
  * Output : out bf16 [B,H,N,d] (rows t >= N are not touched).
- * workspace: at least sagesla_workspace_bytes(shape) bytes. */
+ * workspace: at least sagesla_workspace_bytes(shape) bytes; forward keeps H, Z, z in
+ *          bf16, O_l and the query-block pairing of the attention tiles there. */
 int sagesla_forward(const sagesla_shape* shape, const void* q, float sm_scale,
                     const int8_t* q8, const int8_t* k8, const float* q_scale,
                     const float* k_scale, const void* v, const int32_t* crit_idx, int k_c,
