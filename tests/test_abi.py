@@ -72,6 +72,10 @@ def test_validation_rejects_before_launch(L):
     # unsupported head dim, empty shapes
     assert L.sagesla_counts(ctypes.byref(_sh(d=64)), 0.5, 0.1, ctypes.byref(z), None, None, None) == 2
     assert L.sagesla_counts(ctypes.byref(_sh(N=0)), 0.5, 0.1, None, None, None, None) == 1
+    # limits: at most 8192 blocks of 64 tokens, at most 65535 (batch, head) pairs
+    assert L.sagesla_counts(ctypes.byref(_sh(N=8192 * 64)), 0.5, 0.1, ctypes.byref(z), None, None, None) == 0
+    assert L.sagesla_counts(ctypes.byref(_sh(N=8192 * 64 + 1)), 0.5, 0.1, None, None, None, None) == 2
+    assert L.sagesla_counts(ctypes.byref(_sh(B=2, H=32768)), 0.5, 0.1, None, None, None, None) == 2
     assert L.sagesla_counts(None, 0.5, 0.1, None, None, None, None) == 1
     # null / misaligned device pointers are rejected without touching the GPU
     vp = [None] * 9

@@ -132,7 +132,7 @@ def test_720p_full_size_sampled():
     assert near == 0
 
 
-@pytest.mark.parametrize("rho", [1.0, 0.05])
+@pytest.mark.parametrize("rho", [1.0, 0.5, 0.2, 0.1, 0.05])
 def test_sweep_full_size_sampled(rho):
     near, res = _sampled_check(sweep_workload(rho), heads_for_oracle=1, qblocks_per_head=8, seed=1)
     assert near == 0
@@ -149,3 +149,26 @@ def test_select_large_block_counts(N):
     assert_prepare_bitexact(g, prep)
     assert (g["k_c"], g["n_neg"], g["m"]) == (sel.k_c, sel.n_neg, sel.m)
     assert compare_lists(g, sel) == 0
+
+
+def test_select_at_the_block_limit():
+    # nB = 8192, the largest block count the library accepts (4 query-block rows per CTA).
+    # Rows sampled for the exact check; every row checked for the list structure.
+    N = 8192 * 64
+    q, k, v = make_random_qkv(1, 1, N, seed=8)
+    g = run_gpu_select(q, k, v, 0.1, 0.45)
+    prep = O.prepare(f32(q), f32(k))
+    assert_prepare_bitexact(g, prep)
+    rows = np.sort(np.random.default_rng(0).choice(8192, 12, replace=False))
+    sel = O.select(prep.q_bar[:, :, rows], prep.k_bar, 0.1, 0.45)
+    assert (g["k_c"], g["n_neg"], g["m"]) == (sel.k_c, sel.n_neg, sel.m)
+    np.testing.assert_array_equal(g["logits"][:, :, rows].view(np.uint32), sel.logits.view(np.uint32))
+    np.testing.assert_array_equal(g["crit"][:, :, rows], sel.crit)
+    np.testing.assert_array_equal(g["marg"][:, :, rows], sel.marg)
+    crit, marg, mask = g["crit"][0, 0], g["marg"][0, 0], g["mask"][0, 0]
+    assert (np.diff(crit, axis=1) > 0).all() and (np.diff(marg, axis=1) > 0).all()
+    member = np.zeros((8192, 8192), dtype=np.int8)
+    np.put_along_axis(member, crit.astype(np.int64), 1, axis=1)
+    np.put_along_axis(member, marg.astype(np.int64), 2, axis=1)
+    assert ((member == 1).sum(1) == sel.k_c).all() and ((member == 2).sum(1) == sel.m).all()
+    np.testing.assert_array_equal(mask[:, :8192], (member == 2).astype(np.float32))
