@@ -119,8 +119,9 @@ int sagesla_prepare_static_scratch(const sagesla_shape* shape, const void* q, co
  *          marg_mask bf16 [B,H,nB,nBp]  1.0 where block j is marginal for row i, 0
  *                                       elsewhere (including the pitch padding)
  *          logits   fp32 [B,H,nB,nB]    optional (NULL = not written)
- * Logits use a fixed fp32 order (acc = 0; acc = fl32(acc + fl32(qbar*kbar)) for
- * c = 0..d-1), so the lists are bit-exact against any implementation that follows it. */
+ * Logits use a fixed fp32 order, one fused multiply-add per channel (acc = 0;
+ * acc = fl32(qbar[c]*kbar[c] + acc) for c = 0..d-1), so the lists are bit-exact against
+ * any implementation that follows it. */
 int sagesla_select(const sagesla_shape* shape, const float* q_bar, const float* k_bar,
                    double rho, double nu, int32_t* crit_idx, int32_t* marg_idx,
                    void* marg_mask, float* logits, void* stream);

@@ -248,17 +248,41 @@ class Selection:
         return M
 
 
+def fma32(a, b, c) -> np.ndarray:
+    """fl32(a*b + c) for float32 a, b, c: one rounding, to nearest even (IEEE fusedMultiplyAdd).
+
+    a*b is exact in float64 (24 + 24 bits). p + c is formed in float64 with round-to-odd:
+    the float64 sum s and its exact error e (Knuth's TwoSum) give the odd neighbour of the
+    exact value whenever e != 0. A value rounded to odd in a format with at least 2 more
+    bits than the target (53 >= 24 + 2) rounds to the target exactly as the exact value
+    would (Boldo and Melquiond, "Emulation of FMA and correctly rounded sums: proved
+    algorithms using rounding to odd", IEEE Trans. Computers 57(4), 2008), so the final cast
+    to float32 is the correctly rounded result.
+    """
+    p = np.asarray(a, dtype=np.float64) * np.asarray(b, dtype=np.float64)
+    c = np.asarray(c, dtype=np.float64)
+    s = p + c
+    bb = s - p
+    e = (p - (s - bb)) + (c - bb)
+    bits = s.view(np.int64)
+    even = (bits & 1) == 0
+    fix = (e != 0) & even & np.isfinite(s)
+    s_odd = np.where(fix, np.nextafter(s, np.where(e > 0, np.inf, -np.inf)), s)
+    return s_odd.astype(_F32)
+
+
 def block_logits(q_bar: np.ndarray, k_bar: np.ndarray) -> np.ndarray:
     """l_ij = mean(Q~_i) . mean(K~_j) in fp32.
 
-    Fixed order: acc = +0.0; for c = 0..d-1: acc = fl32(acc + fl32(qbar_i[c] * kbar_j[c])).
+    Fixed order, one fused multiply-add per channel: acc = +0.0; for c = 0..d-1:
+    acc = fl32(qbar_i[c] * kbar_j[c] + acc).
     """
     qb = q_bar.astype(_F32)
     kb = k_bar.astype(_F32)
     B, H, nB, d = qb.shape
     acc = np.zeros((B, H, nB, kb.shape[2]), dtype=_F32)
     for c in range(d):
-        acc = acc + (qb[:, :, :, None, c] * kb[:, :, None, :, c])
+        acc = fma32(qb[:, :, :, None, c], kb[:, :, None, :, c], acc)
     return acc
 
 

@@ -6,12 +6,13 @@
 // the kept fraction (0.1 -> 90% sparsity).
 //
 // One CTA handles R = 2*RT query-block rows of one head (two row groups of 128 threads):
-//   1. l_ij = fp32 dot of the block means in a fixed order (acc = 0; for c: acc =
-//      fl32(acc + fl32(qbar[c]*kbar[c]))) - separate multiply and add, no FMA, so any
+//   1. l_ij = fp32 dot of the block means in a fixed order, one fused multiply-add per
+//      channel (acc = 0; for c = 0..127: acc = fl32(qbar[c]*kbar[c] + acc)), so any
 //      implementation following the order gets the same bits. Each thread keeps an
-//      RT x 4 tile of (row, key block) fp32 accumulators; the key means are staged
-//      channel-major in shared memory, 16 channels at a time, by a double-buffered
-//      cp.async pipeline; the row means are read as broadcasts.
+//      RT x 4 tile of (row, key block) accumulators as packed f32x2 pairs (fma.rn.f32x2:
+//      two correctly rounded FMAs per instruction); the key means are staged
+//      channel-major in shared memory, 8 channels at a time, by a double-buffered
+//      cp.async pipeline; each row mean is stored twice so one load gives a (q, q) pair.
 //   2. Each row's logits become order-preserving 32-bit keys. One warp per row finds the
 //      k_c-th largest key T_c and the n_neg-th smallest key T_n by a most-significant-bit
 //      first search over the key bits (a warp-wide count per bit, stopping as soon as the
@@ -30,12 +31,26 @@ constexpr int kSelThreads = 256;
 constexpr int kGroupThreads = 128;                    // threads per row group (two groups)
 constexpr int kJPerThread = 4;                        // key blocks per thread per pass
 constexpr int kJPass = kGroupThreads * kJPerThread;   // 512 key blocks per pass
-constexpr int kChunk = 16;                            // channels per pipeline stage
+constexpr int kChunk = 8;                             // channels per pipeline stage
 constexpr int kKStride = kJPass + 4;                  // floats per staged channel row
-constexpr int kStages = kHeadDim / kChunk;            // 8 stages per pass
+constexpr int kStages = kHeadDim / kChunk;            // 16 stages per pass
 constexpr int kStageFloats = kChunk * kKStride;
 constexpr int kRegKeysSmall = 16;                     // keys per lane held in registers
 constexpr int kRegKeysLarge = 40;
+
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2_rn(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
 
 struct SelParams {
   const float* qbar;
@@ -55,14 +70,14 @@ __device__ __forceinline__ uint32_t order_key(float l) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Stage channels [c0, c0+16) of key blocks [jbase, jbase+512) channel-major: a half warp
-// reads one block's 64 contiguous bytes, each lane writes one (channel, block) slot.
+// Stage channels [c0, c0+kChunk) of key blocks [jbase, jbase+512) channel-major: kChunk
+// lanes read one block's contiguous channels, each lane writes one (channel, block) slot.
 __device__ __forceinline__ void stage_kbar(const float* kb, float* dst, int jbase, int c0, int nB,
                                            int tid) {
 #pragma unroll 4
   for (int t = 0; t < kJPass * kChunk / kSelThreads; ++t) {
     const int e = tid + t * kSelThreads;
-    const int jj = e >> 4, c = e & (kChunk - 1);
+    const int jj = e / kChunk, c = e % kChunk;
     if (jbase + jj < nB)
       cp_async4(smem_u32(dst + c * kKStride + jj),
                 kb + static_cast<size_t>(jbase + jj) * kHeadDim + c0 + c);
@@ -189,8 +204,8 @@ template <int RT>
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelParams p) {
   constexpr int R = 2 * RT;
   extern __shared__ __align__(16) unsigned char smem[];
-  float* qs = reinterpret_cast<float*>(smem);                 // [R][128] row means
-  float* kT = qs + R * kHeadDim;                              // [2][kChunk][kKStride]
+  float* qd = reinterpret_cast<float*>(smem);                 // [R][2*128] row means, doubled
+  float* kT = qd + R * 2 * kHeadDim;                          // [2][kChunk][kKStride]
   uint32_t* keys = reinterpret_cast<uint32_t*>(kT + 2 * kStageFloats);  // [R][nBk]
 
   const int tid = threadIdx.x, bh = blockIdx.y;
@@ -198,20 +213,20 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelParams p) {
   const int rows = min(R, nB - i0);
   const float* kb = p.kbar + static_cast<size_t>(bh) * nB * kHeadDim;
 
-  for (int x = tid; x < R * kHeadDim / 4; x += kSelThreads) {
-    const int r = x / (kHeadDim / 4);
-    reinterpret_cast<float4*>(qs)[x] =
-        r < rows ? reinterpret_cast<const float4*>(p.qbar + (static_cast<size_t>(bh) * nB + i0) * kHeadDim)[x]
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int x = tid; x < R * kHeadDim / 2; x += kSelThreads) {
+    const int r = x / (kHeadDim / 2);
+    const float2 v = r < rows ? reinterpret_cast<const float2*>(p.qbar + (static_cast<size_t>(bh) * nB + i0) * kHeadDim)[x]
+                              : make_float2(0.f, 0.f);
+    reinterpret_cast<float4*>(qd)[x] = make_float4(v.x, v.x, v.y, v.y);
   }
 
   // ---- 1. logits, 512 key blocks per pass
   const int rg = tid / kGroupThreads, tl = tid % kGroupThreads;
   const int row0 = rg * RT;
   for (int jbase = 0; jbase < nB; jbase += kJPass) {
-    float acc[RT][4];
+    uint64_t acc[RT][2];  // (row, key blocks j0/j0+1) and (row, j0+2/j0+3)
 #pragma unroll
-    for (int r = 0; r < RT; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+    for (int r = 0; r < RT; ++r) acc[r][0] = acc[r][1] = 0ull;  // +0.0f pairs
     const int j0 = jbase + kJPerThread * tl;
     const bool active = j0 < nB;
 
@@ -227,25 +242,22 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelParams p) {
       }
       __syncthreads();
       if (active) {
-        // Separate round-to-nearest multiply and add (never contracted into an FMA).
         const float* kt = kT + (s & 1) * kStageFloats + kJPerThread * tl;
-        const float* qrow = qs + row0 * kHeadDim + s * kChunk;
+        const float* qs = qd + row0 * 2 * kHeadDim + 2 * s * kChunk;
 #pragma unroll
-        for (int c4 = 0; c4 < kChunk; c4 += 4) {
-          float4 kv[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) kv[e] = *reinterpret_cast<const float4*>(kt + (c4 + e) * kKStride);
+        for (int cc = 0; cc < kChunk; cc += 2) {
+          const float4 k0 = *reinterpret_cast<const float4*>(kt + cc * kKStride);
+          const float4 k1 = *reinterpret_cast<const float4*>(kt + (cc + 1) * kKStride);
+          const uint64_t k0a = f2pack(k0.x, k0.y), k0b = f2pack(k0.z, k0.w);
+          const uint64_t k1a = f2pack(k1.x, k1.y), k1b = f2pack(k1.z, k1.w);
 #pragma unroll
           for (int r = 0; r < RT; ++r) {
-            const float4 q = *reinterpret_cast<const float4*>(qrow + r * kHeadDim + c4);
-            const float qc[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {  // channel c4 + e, in order
-              acc[r][0] = __fadd_rn(acc[r][0], __fmul_rn(qc[e], kv[e].x));
-              acc[r][1] = __fadd_rn(acc[r][1], __fmul_rn(qc[e], kv[e].y));
-              acc[r][2] = __fadd_rn(acc[r][2], __fmul_rn(qc[e], kv[e].z));
-              acc[r][3] = __fadd_rn(acc[r][3], __fmul_rn(qc[e], kv[e].w));
-            }
+            const float4 q = *reinterpret_cast<const float4*>(qs + r * 2 * kHeadDim + 2 * cc);
+            const uint64_t qa = f2pack(q.x, q.y), qb = f2pack(q.z, q.w);  // (q_c, q_c), (q_c+1, q_c+1)
+            acc[r][0] = fma2_rn(qa, k0a, acc[r][0]);  // channel c
+            acc[r][1] = fma2_rn(qa, k0b, acc[r][1]);
+            acc[r][0] = fma2_rn(qb, k1a, acc[r][0]);  // channel c + 1
+            acc[r][1] = fma2_rn(qb, k1b, acc[r][1]);
           }
         }
       }
@@ -257,7 +269,9 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelParams p) {
       for (int r = 0; r < RT; ++r) {
         const int row = row0 + r;
         if (row < rows) {
-          const float* l = acc[r];
+          float l[4];
+          f2unpack(acc[r][0], l[0], l[1]);
+          f2unpack(acc[r][1], l[2], l[3]);
           uint4 kv;
           kv.x = order_key(l[0]);
           kv.y = j0 + 1 < nB ? order_key(l[1]) : 0u;
@@ -293,7 +307,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelParams p) {
 template <int RT>
 cudaError_t launch_rt(const Dims& g, const SelParams& p, cudaStream_t st) {
   constexpr int R = 2 * RT;
-  const size_t smem = static_cast<size_t>(R) * kHeadDim * 4 +
+  const size_t smem = static_cast<size_t>(R) * 2 * kHeadDim * 4 +
                       static_cast<size_t>(2) * kStageFloats * 4 +
                       static_cast<size_t>(R) * p.nBk * 4;
   cudaError_t e = cudaFuncSetAttribute(select_kernel<RT>,

@@ -120,6 +120,51 @@ def test_block_means_close_to_numpy():
 
 
 # ------------------------------------------------------------------ step 4: selection
+def _rn32(x):
+    """Round an exact rational to the nearest float32, ties to even (normal and subnormal)."""
+    from fractions import Fraction
+    if x == 0:
+        return np.float32(0.0)
+    sign = -1 if x < 0 else 1
+    x = abs(x)
+    e = x.numerator.bit_length() - x.denominator.bit_length()
+    while Fraction(2) ** e > x:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= x:
+        e += 1
+    q = max(e, -126) - 23
+    m = x / Fraction(2) ** q
+    n = m.numerator // m.denominator
+    r = m - n
+    if r > Fraction(1, 2) or (r == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return np.float32(float(sign * n * Fraction(2) ** q))
+
+
+def test_fma32_is_correctly_rounded():
+    # The block logits are a chain of fp32 fused multiply-adds: fl32(a*b + c), one rounding.
+    # Checked against exact rational arithmetic on random and cancelling operands, and on a
+    # case where rounding a*b + c to float64 first and then to float32 (double rounding)
+    # gives the wrong answer: a*b + c = 1 + 3*2^-24 - 2^-70 lies just below a float32
+    # midpoint, its float64 rounding lands on the midpoint, and ties-to-even then rounds up.
+    from fractions import Fraction
+    rng = np.random.default_rng(1)
+    n = 3000
+    a = (rng.standard_normal(n) * np.exp2(rng.integers(-20, 20, n))).astype(np.float32)
+    b = (rng.standard_normal(n) * np.exp2(rng.integers(-20, 20, n))).astype(np.float32)
+    p32 = (a.astype(np.float64) * b).astype(np.float32)
+    c = np.where(rng.random(n) < 0.5, (-p32 * (1 + rng.integers(-3, 4, n) * 2.0 ** -23)).astype(np.float32),
+                 (rng.standard_normal(n) * np.exp2(rng.integers(-20, 20, n))).astype(np.float32))
+    a = np.append(a, np.float32(1 + 2.0 ** -23))
+    b = np.append(b, np.float32(2.0 ** -24 * (1 - 2.0 ** -23)))
+    c = np.append(c, np.float32(1 + 2.0 ** -23))
+    exact = np.array([_rn32(Fraction(float(x)) * Fraction(float(y)) + Fraction(float(z)))
+                      for x, y, z in zip(a, b, c)], dtype=np.float32)
+    np.testing.assert_array_equal(O.fma32(a, b, c).view(np.uint32), exact.view(np.uint32))
+    naive = (a.astype(np.float64) * b + c).astype(np.float32)
+    assert naive[-1] != exact[-1]  # the planted case separates the two
+
+
 def test_logits_close_to_fp64_dot():
     rng = np.random.default_rng(5)
     qb = rng.normal(size=(1, 2, 9, 128)).astype(np.float32)
