@@ -6,19 +6,26 @@
 // Sparse-Linear Attention - SLA" (exact attention only on the selected block pairs; the
 // two stack as "SageSLA").
 //
-// Design (sm_100a):
-//   * One CTA owns a PAIR of adjacent 64-row query blocks, i.e. one 128-row tile, so every
-//     tensor-core instruction is a full M = 128 tcgen05.mma. The CTA walks the union of
-//     the two blocks' ascending critical lists; for a key block in only one list the other
-//     half's rows are masked (their P row is 0). Adjacent query blocks share most critical
-//     key blocks, which also halves the K/V traffic per query row.
-//   * Warp-specialised: warp 0 issues TMA loads (Q8 pair once; per union step one INT8 K
-//     tile and one bf16 V tile into a 4-stage ring), warp 1 issues tcgen05.mma (kind::i8
-//     S = Q8 K8^T into one of two TMEM S buffers; kind::f16 O += P V into TMEM), warps 2-5
-//     run the online softmax: one thread per query row, scores dequantised by
-//     s_q * s_k * log2(e), exp2 on the SFU, P rounded to bf16 into shared memory (the A
-//     operand of the P V MMA). The running max is raised only when a tile's max exceeds
-//     it by more than 8 (in log2 units), so the O rescale in TMEM is rare.
+// Design (sm_100a), two CTAs per SM:
+//   * One CTA owns a PAIR of 64-row query blocks, i.e. one 128-row tile, so every
+//     tensor-core instruction is a full M = 128 tcgen05.mma. pair_kernel chooses the
+//     pairs: blocks sharing many critical key blocks go together. The CTA walks the union
+//     of the two blocks' ascending critical lists; for a key block in only one list the
+//     P.V MMA masks the other half's rows (disable-output-lane mask).
+//   * Warp-specialised:
+//     - warp 0, TMA producer: the pair's Q8 once; per union step one INT8 K tile (8 KB)
+//       into a 5-slot ring (with the step's block index, membership and k-scale beside
+//       it) and one bf16 V tile (16 KB) into a 3-slot ring.
+//     - warp 1, one thread issues every tcgen05.mma: kind::i8 S = Q8 K8^T (M128 N64 K128,
+//       s32) into one of two 64-column TMEM score buffers, then kind::f16 O += P V with P
+//       read from TMEM (M128 N128 K64, fp32 O in TMEM). QK(t+1) is issued before waiting
+//       for P(t); P.V(t) as soon as the member halves have written P(t).
+//     - warps 2-9, softmax: two threads per query row (16-lane TMEM shapes, 16 keys each
+//       of two rows), scores dequantised by s_q * s_k * log2(e) through an exact
+//       magic-number int->float and packed f32x2 FMAs, exp2 on the SFU, P rounded to bf16
+//       and written over the row's score columns.
+//   * The running max m is raised only when a tile's partial sum of 2^(s - m) leaves
+//     [0, 2^24]; only then is the exact tile max taken and O rescaled in TMEM.
 //   * Epilogue: O_s = O / l, plus the linear-branch O_l, rounded once to bf16.
 // Every mbarrier wait is bounded (see sm100_primitives.cuh) and never traps.
 #include <climits>

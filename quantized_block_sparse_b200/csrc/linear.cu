@@ -9,13 +9,14 @@
 //
 // Kernels:
 //   hgemm_kernel   H = M . h per head, M the 0/1 marginal mask [nB x nBp] and h viewed as
-//                  [nB x d*d]: a tcgen05 bf16 GEMM (fp32 accumulation in TMEM), 128x128
-//                  output tiles, TMA-fed 3-stage pipeline, bf16 output.
+//                  [nB x d*d]: a persistent tcgen05 bf16 GEMM (fp32 accumulation in two
+//                  TMEM accumulators), 128x256 output tiles, TMA-fed 4-stage pipeline,
+//                  bf16 output; plus one 128-column tile for Z.
 //   zb_kernel      z_j rounded to bf16; hgemm_kernel's extra column tile gives Z = M . z
 //                  (bf16 operands, fp32 accumulation and output, like H).
-//   linout_kernel  per pair of query blocks: phi(Q~) (recomputed from Q, bf16) times H_i
-//                  on tcgen05 (M = 128 rows = both blocks, one MMA chain per block),
-//                  divided by phi(Q~) . Z_i; bf16 O_l for the attention epilogue.
+//   linout_kernel  per pair of adjacent query blocks: phi(Q~) (recomputed from Q, bf16)
+//                  times H_i on tcgen05 (M = 128 rows = both blocks, one MMA chain per
+//                  block), divided by phi(Q~) . Z_i; bf16 O_l for the attention epilogue.
 #include "sagesla_internal.h"
 #include "sm100_primitives.cuh"
 
