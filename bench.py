@@ -43,10 +43,12 @@ def dense_equiv_ops(wl) -> float:
 def profiled_traffic(workload: str):
     """DRAM bytes per attn_kernel launch from the committed ncu summary, or None.
 
-    The summary records the sha256 prefix of the kernel source it was taken on; once the
-    source has changed the counters no longer describe the kernel and None is returned.
+    The summary records the sha256 prefix of the kernel source it was taken on (comments
+    and whitespace removed, so only code counts); once the code has changed the counters
+    no longer describe the kernel and None is returned.
     """
     import hashlib
+    import re
     summary = os.path.join(ROOT, "profiles", f"attn_kernel_{workload}.md")
     src = os.path.join(ROOT, "quantized_block_sparse_b200", "csrc", "attention.cu")
     if not (os.path.exists(summary) and os.path.exists(src)):
@@ -57,8 +59,12 @@ def profiled_traffic(workload: str):
             if ":" in line and not line.startswith(("|", "#", " ")):
                 key, _, val = line.partition(":")
                 fields[key.strip()] = val.strip()
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
+    with open(src) as f:
+        code = f.read()
+    code = re.sub(r"/\*.*?\*/", " ", code, flags=re.S)
+    code = re.sub(r"//[^\n]*", " ", code)
+    code = re.sub(r"\s+", " ", code).strip()
+    sha = hashlib.sha256(code.encode()).hexdigest()
     prefix = fields.get("source_sha256_prefix")
     if not prefix or not sha.startswith(prefix) or "dram_bytes_per_launch" not in fields:
         return None
