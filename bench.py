@@ -254,6 +254,26 @@ def whole_job_tops(ops_per_rank: float, world: int, step_ms: float) -> float:
     return ops_per_rank * world / (step_ms * 1e-3) / 1e12
 
 
+def gpu_local_cpus(device_index: int):
+    """The CPUs NVML reports as local to the GPU (its NUMA node), or None."""
+    try:
+        import pynvml
+        import torch
+        pr = torch.cuda.get_device_properties(device_index)
+        bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+        pynvml.nvmlInit()
+        try:
+            handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            words = pynvml.nvmlDeviceGetCpuAffinity(handle, (os.cpu_count() + 63) // 64)
+        finally:
+            pynvml.nvmlShutdown()
+        cpus = {64 * i + b for i, w in enumerate(words) for b in range(64) if (w >> b) & 1}
+        cpus &= os.sched_getaffinity(0)
+        return cpus or None
+    except Exception:
+        return None
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_ours(args, wl):
     import torch
@@ -328,8 +348,19 @@ def run_ours(args, wl):
     # input sets and two output buffers; host->device and device->host overlap). Every
     # step's copies are inside the timed region, which ends when the last output has
     # reached the host.
-    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
-    ohs = [torch.empty_like(q).pin_memory() for _ in range(2)]
+    # Pinned host buffers on the GPU's NUMA node (allocated while the process runs on the
+    # GPU-local CPUs; the previous CPU set is restored afterwards).
+    local_cpus = gpu_local_cpus(local)
+    saved_cpus = os.sched_getaffinity(0)
+    if local_cpus:
+        os.sched_setaffinity(0, local_cpus)
+    try:
+        qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+        ohs = [torch.empty_like(q).pin_memory() for _ in range(2)]
+        for t in ohs:
+            t.zero_()
+    finally:
+        os.sched_setaffinity(0, saved_cpus)
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = ohs[0].numel() * ohs[0].element_size()
     ins = [(qd, kd, vd), tuple(torch.empty_like(t) for t in (qd, kd, vd))]
@@ -403,7 +434,8 @@ def run_ours(args, wl):
                               f"traffic = DRAM bytes per launch from the committed ncu summary "
                               f"(null once the kernel source differs from the profiled one)")},
         "e2e": {"value": whole_job_tops(dense_equiv_ops(wl), world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "pinned_host_memory": "GPU-local NUMA node" if local_cpus else "default placement"},
         "gpu_launches": int(round(launches_per_step * args.steps)),
         "clocks": clk,
     }
