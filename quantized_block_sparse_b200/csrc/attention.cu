@@ -592,12 +592,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           }
         };
         run_tile();
-        // rare path: raise m where a partial sum left [0, 2^24] (quad-consistent decision)
-        bool need0 = !(ps0 <= kPsumLimit), need1 = !(ps1 <= kPsumLimit);
-        need0 = quad_any(need0);
-        need1 = quad_any(need1);
+        // rare path: raise m where a partial sum left [0, 2^24] (quad-consistent decision;
+        // the warp-wide test first keeps the common path to one vote)
         float alpha0 = 1.f, alpha1 = 1.f;
-        if (__any_sync(0xffffffffu, need0 || need1)) {
+        bool rescale = false;
+        if (__any_sync(0xffffffffu, !(ps0 <= kPsumLimit) || !(ps1 <= kPsumLimit))) {
+          const bool need0 = quad_any(!(ps0 <= kPsumLimit)), need1 = quad_any(!(ps1 <= kPsumLimit));
           // S_b still holds the scores (P overwrites it only below): reload them.
           tmem_ld_16x256b_x8(taddr + lane_off + 64 * b, sv);
 #pragma unroll
@@ -628,11 +628,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             m1 = mt;
           }
           run_tile();
+          rescale = __any_sync(0xffffffffu, alpha0 != 1.f || alpha1 != 1.f);
         }
         l0 = fmaf(l0, alpha0, ps0);
         l1 = fmaf(l1, alpha1, ps1);
         tmem_st_16x128b_x8(taddr + lane_off + 64 * b, pk);  // P first: its registers die here
-        if (__any_sync(0xffffffffu, alpha0 != 1.f || alpha1 != 1.f)) {
+        if (rescale) {  // warp-uniform
           // O holds P.V of earlier steps: wait for the last issued P.V, then rescale rows.
           if (t >= 1)
             ok = mbar_wait(smem_u32(pv_done + ((t - 1) & 1)), ((t - 1) >> 1) & 1, &abort_flag,
