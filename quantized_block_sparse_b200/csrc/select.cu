@@ -5,22 +5,27 @@
 // covers the middle and the rest is skipped; section "Hands-On Tutorial": --sla_topk sets
 // the kept fraction (0.1 -> 90% sparsity).
 //
-// One CTA handles R = 2*RT query-block rows of one head (two row groups of 128 threads):
+// One CTA handles R = 2*RT query-block rows of one head (two row groups of 128 threads);
+// R is the largest of 22, 16, 12, 8, 4 whose keys still let two CTAs share an SM:
 //   1. l_ij = fp32 dot of the block means in a fixed order, one fused multiply-add per
 //      channel (acc = 0; for c = 0..127: acc = fl32(qbar[c]*kbar[c] + acc)), so any
 //      implementation following the order gets the same bits. Each thread keeps an
 //      RT x 4 tile of (row, key block) accumulators as packed f32x2 pairs (fma.rn.f32x2:
 //      two correctly rounded FMAs per instruction); the key means are staged
-//      channel-major in shared memory, 8 channels at a time, by a double-buffered
-//      cp.async pipeline; each row mean is stored twice so one load gives a (q, q) pair.
+//      channel-major in shared memory, 8 channels at a time: 16-byte global loads run one
+//      stage ahead in registers and are transposed into two alternating slots by 4-byte
+//      stores, one barrier per stage; each row mean is stored twice so one load gives a
+//      (q, q) pair.
 //   2. Each row's logits become order-preserving 32-bit keys. One warp per row finds the
-//      k_c-th largest key T_c and the n_neg-th smallest key T_n by a most-significant-bit
-//      first search over the key bits (a warp-wide count per bit, stopping as soon as the
-//      count is exactly k_c). Total order: logit descending, block index ascending.
+//      k_c-th largest key T_c and the n_neg-th smallest key T_n by most-significant-bit
+//      first searches over the key bits, both in one loop (one warp-wide reduction per bit
+//      carries both counts), each stopping as soon as its count is exact. Total order:
+//      logit descending, block index ascending.
 //   3. Critical: key > T_c, plus the lowest-index blocks with key == T_c up to k_c in
 //      all. Negligible: key < T_n, plus the highest-index blocks with key == T_n up to
 //      n_neg. The rest is marginal. A warp-ballot compaction writes both lists in
-//      ascending block order and the 0/1 bf16 marginal mask row.
+//      ascending block order and the 0/1 bf16 marginal mask row; the per-tie ballots run
+//      only when a threshold splits a run of equal keys.
 #include "sagesla_internal.h"
 #include "sm100_primitives.cuh"
 
@@ -70,17 +75,34 @@ __device__ __forceinline__ uint32_t order_key(float l) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Stage channels [c0, c0+kChunk) of key blocks [jbase, jbase+512) channel-major: kChunk
-// lanes read one block's contiguous channels, each lane writes one (channel, block) slot.
-__device__ __forceinline__ void stage_kbar(const float* kb, float* dst, int jbase, int c0, int nB,
+// Channels [c0, c0+kChunk) of key blocks [jbase, jbase+512): four 16-byte global loads per
+// thread (float4 f holds channels c0+4*(f%2) .. +3 of block f/2), held in registers one
+// stage ahead of use; blocks at or past nB read as zeros.
+__device__ __forceinline__ void load_stage(const float* kb, float4 (&v)[4], int jbase, int c0, int nB,
                                            int tid) {
-#pragma unroll 4
-  for (int t = 0; t < kJPass * kChunk / kSelThreads; ++t) {
-    const int e = tid + t * kSelThreads;
-    const int jj = e / kChunk, c = e % kChunk;
-    if (jbase + jj < nB)
-      cp_async4(smem_u32(dst + c * kKStride + jj),
-                kb + static_cast<size_t>(jbase + jj) * kHeadDim + c0 + c);
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int f = tid + t * kSelThreads;
+    const int jj = f >> 1, g = f & 1;
+    v[t] = jbase + jj < nB
+               ? __ldg(reinterpret_cast<const float4*>(kb + static_cast<size_t>(jbase + jj) * kHeadDim + c0 + 4 * g))
+               : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// Transpose a loaded stage into its channel-major slot with 4-byte stores: for each of the
+// four channels, the 32 lanes of a warp hit 16 consecutive blocks in two channel rows whose
+// bank offsets differ by 16, so every store is conflict-free.
+__device__ __forceinline__ void store_stage(float* dst, const float4 (&v)[4], int tid) {
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int f = tid + t * kSelThreads;
+    const int jj = f >> 1, g = f & 1;
+    float* d = dst + 4 * g * kKStride + jj;
+    d[0] = v[t].x;
+    d[kKStride] = v[t].y;
+    d[2 * kKStride] = v[t].z;
+    d[3 * kKStride] = v[t].w;
   }
 }
 
@@ -126,59 +148,114 @@ __device__ __forceinline__ int warp_count(const RowKeys<KPL>& K, Pred pred) {
   return __reduce_add_sync(0xffffffffu, c);
 }
 
+// Two warp-wide counts in one reduction: low half #pred_lo, high half #pred_hi. A row has
+// at most 8192 keys, so neither half overflows into the other.
+template <int KPL, class PredLo, class PredHi>
+__device__ __forceinline__ void warp_count2(const RowKeys<KPL>& K, PredLo lo, PredHi hi, int& c_lo,
+                                            int& c_hi) {
+  uint32_t c = 0;
+  if constexpr (KPL > 0) {
+#pragma unroll
+    for (int t = 0; t < KPL; ++t) c += (lo(K.v[t]) ? 1u : 0u) + (hi(K.v[t]) ? 0x10000u : 0u);
+  } else {
+    for (int t = 0; t < K.nt; ++t) {
+      const uint32_t x = K.at(t);
+      c += (lo(x) ? 1u : 0u) + (hi(x) ? 0x10000u : 0u);
+    }
+  }
+  c = __reduce_add_sync(0xffffffffu, c);
+  c_lo = static_cast<int>(c & 0xffffu);
+  c_hi = static_cast<int>(c >> 16);
+}
+
 // Classify one row and write its lists and mask row (one warp, warp-uniform control).
+//
+// T_c, the k_c-th largest key, is the largest T with #{key >= T} >= k_c. The n_neg-th
+// smallest valid key is T_n = ~U for the largest U with #{1 <= key <= ~U} >= n_neg; since
+// key <= ~U is key < -U (two's complement, U >= 1) and empty slots hold 0, that count is
+// nB - #{key >= -U}. Both are found bit by bit from the most significant bit, in one loop
+// while both are open (one reduction per bit for the two counts); a search stops as soon as
+// its count is exactly its target, because then no later bit can change the split.
 template <int KPL>
 __device__ void classify_row(const SelParams& p, const uint32_t* kr, size_t row, int lane) {
   RowKeys<KPL> K;
   K.load(kr, p.nB, p.nBp, lane);
-  const int k_c = p.k_c, n_neg = p.n_neg;
+  const int k_c = p.k_c, n_neg = p.n_neg, nB = p.nB;
 
-  // k_c-th largest key: the largest T with #{key >= T} >= k_c.
-  uint32_t Tc = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = Tc | (1u << bit);
-    const int c = warp_count(K, [cand](uint32_t x) { return x >= cand; });
-    if (c >= k_c) {
-      Tc = cand;
-      if (c == k_c) break;  // {key >= cand} is exactly the critical set
+  uint32_t Tc = 0, U = 0;
+  bool done_c = false, done_n = n_neg <= 0;
+  int bit = 31;
+  for (; bit >= 0 && !done_c && !done_n; --bit) {
+    const uint32_t cc = Tc | (1u << bit), cn = U | (1u << bit), tn = 0u - cn;
+    int gc, gn;
+    warp_count2(K, [cc](uint32_t x) { return x >= cc; }, [tn](uint32_t x) { return x >= tn; }, gc,
+                gn);
+    if (gc >= k_c) {
+      Tc = cc;
+      done_c = gc == k_c;
+    }
+    if (nB - gn >= n_neg) {
+      U = cn;
+      done_n = nB - gn == n_neg;
     }
   }
-  const int need_c = k_c - warp_count(K, [Tc](uint32_t x) { return x > Tc; });
+  for (; bit >= 0 && !done_c; --bit) {
+    const uint32_t cc = Tc | (1u << bit);
+    const int gc = warp_count(K, [cc](uint32_t x) { return x >= cc; });
+    if (gc >= k_c) {
+      Tc = cc;
+      done_c = gc == k_c;
+    }
+  }
+  for (; bit >= 0 && !done_n; --bit) {
+    const uint32_t cn = U | (1u << bit), tn = 0u - cn;
+    const int gn = warp_count(K, [tn](uint32_t x) { return x >= tn; });
+    if (nB - gn >= n_neg) {
+      U = cn;
+      done_n = nB - gn == n_neg;
+    }
+  }
 
-  // n_neg-th smallest key, searched as the n_neg-th largest complemented key; empty
-  // slots (0) are excluded by testing 1 <= key <= X as (key - 1) < X.
-  uint32_t Tn = 0;
+  // Ties at a threshold: critical takes the lowest-index keys equal to T_c, negligible the
+  // highest-index keys equal to T_n. Only a split inside a run of ties needs the ballots.
+  int gt_c, eq_c;
+  warp_count2(K, [Tc](uint32_t x) { return x > Tc; }, [Tc](uint32_t x) { return x == Tc; }, gt_c,
+              eq_c);
+  const int need_c = k_c - gt_c;
+  const uint32_t Tn = ~U;
   int need_n = 0, eq_n = 0;
   if (n_neg > 0) {
-    uint32_t T = 0;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = T | (1u << bit), X = ~cand;
-      const int c = warp_count(K, [X](uint32_t x) { return x - 1u < X; });
-      if (c >= n_neg) {
-        T = cand;
-        if (c == n_neg) break;
-      }
-    }
-    Tn = ~T;
-    need_n = n_neg - warp_count(K, [Tn](uint32_t x) { return x - 1u < Tn - 1u; });
-    eq_n = warp_count(K, [Tn](uint32_t x) { return x == Tn; });
+    int lt_n;
+    warp_count2(K, [Tn](uint32_t x) { return x - 1u < Tn - 1u; },
+                [Tn](uint32_t x) { return x == Tn; }, lt_n, eq_n);
+    need_n = n_neg - lt_n;
   }
+  const bool split_c = need_c > 0 && need_c < eq_c;
+  const bool all_c = need_c > 0 && need_c >= eq_c;
+  const bool split_n = need_n > 0 && need_n < eq_n;
+  const bool all_n = need_n > 0 && need_n >= eq_n;
 
   const unsigned lt = (1u << lane) - 1u;
   int nc = 0, nm = 0, seen_c = 0, seen_n = 0;
   auto chunk = [&](int t, uint32_t key) {
     const int j = 32 * t + lane;
-    const bool valid = j < p.nB;
-    const bool eqc = valid && key == Tc;
-    const unsigned be = __ballot_sync(0xffffffffu, eqc);
-    const bool isc = valid && (key > Tc || (eqc && seen_c + __popc(be & lt) < need_c));
-    seen_c += __popc(be);
+    const bool valid = j < nB;
+    bool isc = valid && (key > Tc || (all_c && key == Tc));
+    if (split_c) {
+      const bool eqc = valid && key == Tc;
+      const unsigned be = __ballot_sync(0xffffffffu, eqc);
+      isc = isc || (eqc && seen_c + __popc(be & lt) < need_c);
+      seen_c += __popc(be);
+    }
     bool isn = false;
     if (n_neg > 0) {
-      const bool eqn = valid && key == Tn;
-      const unsigned bn = __ballot_sync(0xffffffffu, eqn);
-      isn = valid && (key < Tn || (eqn && seen_n + __popc(bn & lt) >= eq_n - need_n));
-      seen_n += __popc(bn);
+      isn = valid && (key < Tn || (all_n && key == Tn));
+      if (split_n) {
+        const bool eqn = valid && key == Tn;
+        const unsigned bn = __ballot_sync(0xffffffffu, eqn);
+        isn = isn || (eqn && seen_n + __popc(bn & lt) >= eq_n - need_n);
+        seen_n += __popc(bn);
+      }
     }
     const bool ism = valid && !isc && !isn;
     const unsigned bc = __ballot_sync(0xffffffffu, isc);
@@ -220,7 +297,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelParams p) {
     reinterpret_cast<float4*>(qd)[x] = make_float4(v.x, v.x, v.y, v.y);
   }
 
-  // ---- 1. logits, 512 key blocks per pass
+  // ---- 1. logits, 512 key blocks per pass; channel stages alternate between two slots
   const int rg = tid / kGroupThreads, tl = tid % kGroupThreads;
   const int row0 = rg * RT;
   for (int jbase = 0; jbase < nB; jbase += kJPass) {
@@ -230,16 +307,14 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelParams p) {
     const int j0 = jbase + kJPerThread * tl;
     const bool active = j0 < nB;
 
-    stage_kbar(kb, kT, jbase, 0, nB, tid);
-    cp_async_commit();
+    float4 ahead[4];
+    load_stage(kb, ahead, jbase, 0, nB, tid);
     for (int s = 0; s < kStages; ++s) {
-      if (s + 1 < kStages) {
-        stage_kbar(kb, kT + ((s + 1) & 1) * kStageFloats, jbase, (s + 1) * kChunk, nB, tid);
-        cp_async_commit();
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
+      // Slot s%2 was last read at stage s-2, which every thread finished before the barrier
+      // of stage s-1; the barrier below publishes the slot. Stage s+1's loads stay in flight
+      // across the barrier and this stage's arithmetic.
+      store_stage(kT + (s & 1) * kStageFloats, ahead, tid);
+      if (s + 1 < kStages) load_stage(kb, ahead, jbase, (s + 1) * kChunk, nB, tid);
       __syncthreads();
       if (active) {
         const float* kt = kT + (s & 1) * kStageFloats + kJPerThread * tl;
@@ -261,8 +336,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelParams p) {
           }
         }
       }
-      __syncthreads();
     }
+    __syncthreads();  // every read of this pass's slots precedes the next pass's stores
 
     if (active) {
 #pragma unroll
@@ -304,12 +379,18 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelParams p) {
   }
 }
 
+constexpr size_t kSmemTwoPerSM = 115712;    // (228 KB per SM - 2 x 1 KB reserved) / 2
+constexpr size_t kSmemOnePerSM = 232448;    // 227 KB, the per-CTA opt-in limit
+
+size_t select_smem(int RT, int nBk) {
+  const size_t R = 2 * static_cast<size_t>(RT);
+  return R * 2 * kHeadDim * 4 + 2 * static_cast<size_t>(kStageFloats) * 4 + R * nBk * 4;
+}
+
 template <int RT>
 cudaError_t launch_rt(const Dims& g, const SelParams& p, cudaStream_t st) {
   constexpr int R = 2 * RT;
-  const size_t smem = static_cast<size_t>(R) * 2 * kHeadDim * 4 +
-                      static_cast<size_t>(2) * kStageFloats * 4 +
-                      static_cast<size_t>(R) * p.nBk * 4;
+  const size_t smem = select_smem(RT, p.nBk);
   cudaError_t e = cudaFuncSetAttribute(select_kernel<RT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -339,11 +420,16 @@ cudaError_t launch_select(const Dims& g, const float* q_bar, const float* k_bar,
   p.k_c = k_c;
   p.n_neg = n_neg;
   p.m = m;
-  // Rows per CTA shrink with nB so that the keys of all rows fit in shared memory
-  // (R * nBk * 4 bytes <= 128 KB).
-  if (g.nB <= 2048) return launch_rt<8>(g, p, st);
-  if (g.nB <= 4096) return launch_rt<4>(g, p, st);
-  if (g.nB <= 8192) return launch_rt<2>(g, p, st);
+  // Rows per CTA: the most (2 x 11, 8, 4 or 2) that still lets two CTAs share an SM with
+  // the keys of all rows in shared memory; past that, the most that fit one CTA. Every CTA
+  // stages the head's whole key-mean table, so fewer, taller CTAs cost less. 12 rows were
+  // measured slower than 8: four of the eight warps then classify two rows, four only one.
+  for (const size_t cap : {kSmemTwoPerSM, kSmemOnePerSM}) {
+    if (select_smem(11, p.nBk) <= cap) return launch_rt<11>(g, p, st);
+    if (select_smem(8, p.nBk) <= cap) return launch_rt<8>(g, p, st);
+    if (select_smem(4, p.nBk) <= cap) return launch_rt<4>(g, p, st);
+    if (select_smem(2, p.nBk) <= cap) return launch_rt<2>(g, p, st);
+  }
   return cudaErrorInvalidValue;
 }
 

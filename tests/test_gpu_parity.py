@@ -140,8 +140,8 @@ def test_sweep_full_size_sampled(rho):
 
 @pytest.mark.parametrize("N", [90000, 140000, 270000])
 def test_select_large_block_counts(N):
-    # nB = 1407: row keys read from shared memory instead of registers; nB = 2188 and
-    # 4219: 8 and 4 query-block rows per CTA. Prepare and select only.
+    # nB = 1407: row keys read from shared memory instead of registers; nB = 1407 and 2188:
+    # 8 query-block rows per CTA, 4219: 4. Prepare and select only.
     q, k, v = make_random_qkv(1, 1, N, seed=N)
     g = run_gpu_select(q, k, v, 0.1, 0.45)
     prep = O.prepare(f32(q), f32(k))
