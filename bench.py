@@ -339,7 +339,8 @@ def run_ours(args, wl):
         kern[name] = {"launches": int(cnt), "avg_ms": float(tot) / int(cnt)}
         launches += int(cnt)
     launches_per_step = launches / args.steps
-    fwd_kernels = ("hgemm_kernel", "zsum_kernel", "linout_kernel", "attn_kernel")
+    # the launches of sagesla_forward (S5-S8)
+    fwd_kernels = ("zb_kernel", "hgemm_kernel", "linout_kernel", "pair_kernel", "attn_kernel")
     fwd_ms = sum(kern[n]["avg_ms"] * kern[n]["launches"] / args.steps for n in fwd_kernels if n in kern)
 
     # ---- end to end through the public API: pinned host inputs in, output back to host.
