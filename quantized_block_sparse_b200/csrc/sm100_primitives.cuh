@@ -108,21 +108,6 @@ __device__ __forceinline__ void mbar_wait_inflight(uint32_t bar, uint32_t parity
   mbar_wait(bar, parity, &never, status);
 }
 
-// ---------------------------------------------------------------- cp.async (LDGSTS)
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // ---------------------------------------------------------------- proxy fences
 // Generic-proxy writes to shared memory -> visible to the async proxy (TMA, tcgen05.mma).
 __device__ __forceinline__ void fence_async_smem() {
