@@ -32,7 +32,8 @@ from quantized_block_sparse_b200.inputs import WORKLOADS, make_workload_qkv  # n
 
 METRIC = "SageSLA fwd ms/call & dense-equiv TOPS at Wan-1.3B 480p shape; % tensor roofline"
 UNIT = "dense-equiv TOPS"
-INT8_TO_BF16_RATE = 2.0  # nominal dense INT8 : BF16 tensor rate on B200 (4.5 : 2.25 POPS)
+INT8_TO_BF16_RATE = 2.0  # dense INT8 : BF16 tensor rate on B200: nominal 4.5 : 2.25 POPS;
+                         # a tcgen05 M128 N128 issue-rate probe gave 8124 : 4064 MAC/clk/SM
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
