@@ -9,7 +9,7 @@ Prints one JSON line on rank 0. Multi-GPU (torchrun): every rank runs an indepen
 replica of the workload (the path has no exchange step); the step time is the max over
 ranks and `value` counts the work of all ranks.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 480p|720p|dense|tiny]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 480p|720p|480p_14b|480p_topk015|dense|tiny]
   python bench.py --impl reference ...   # the CPU oracle on a bounded sample (rank 0)
 """
 from __future__ import annotations
@@ -162,8 +162,18 @@ def run_reference(args, wl):
     return 0
 
 
+WORKLOAD_TITLES = {
+    "480p": "Wan-1.3B 480p-shaped SageSLA layer",
+    "720p": "Wan-14B 720p-shaped SageSLA layer",
+    "480p_14b": "Wan2.1-14B 480p-shaped SageSLA layer",
+    "480p_topk015": "Wan-1.3B 480p-shaped SageSLA layer, sla_topk 0.15",
+    "dense": "dense SageSLA test layer (rho = 1)",
+    "tiny": "tiny SageSLA test layer",
+}
+
+
 def workload_config(wl):
-    return {"workload": f"Wan-{'1.3B 480p' if wl.name == '480p' else wl.name}-shaped SageSLA layer",
+    return {"workload": WORKLOAD_TITLES.get(wl.name, f"{wl.name} SageSLA layer"),
             "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "grid_thw": list(wl.grid),
             "rho": wl.rho, "nu": wl.nu, "block": 64, "seed": wl.seeds[0],
             "l2": "no flush; per-step working set ~1.2 GB (inputs 300 MB + states) exceeds the 126 MB L2",

@@ -50,13 +50,17 @@ class Workload:
         return t * h * w
 
 
-# The five workloads used for parity and measurement. Shapes follow the Wan latent
-# grids (480p: 21x30x52 tokens, 720p: 21x45x80) with head dim 128.
+# Workloads for parity and measurement. Shapes follow the Wan latent grids (480p:
+# 21x30x52 tokens, 720p: 21x45x80) with head dim 128: the 1.3B model has 12 heads, the
+# 14B models 40. "480p_14b" (Wan2.1-14B at 480p) and "480p_topk015" (--sla_topk 0.15 on
+# the 1.3B layer) are second workloads on the same kernels.
 WORKLOADS = {
     "tiny": Workload("tiny", 1, 2, (4, 16, 16), 0.25, 0.25),
     "dense": Workload("dense", 1, 12, (4, 32, 32), 1.0, 0.0),
     "480p": Workload("480p", 1, 12, (21, 30, 52), 0.10, 0.45),
     "720p": Workload("720p", 1, 40, (21, 45, 80), 0.10, 0.45),
+    "480p_14b": Workload("480p_14b", 1, 40, (21, 30, 52), 0.10, 0.45),
+    "480p_topk015": Workload("480p_topk015", 1, 12, (21, 30, 52), 0.15, 0.45),
 }
 SWEEP_RHOS = (1.0, 0.5, 0.2, 0.1, 0.05)
 
