@@ -5,9 +5,9 @@ One step = one pass of the whole path over one batch of synthetic input: sagesla
 sagesla_select and sagesla_forward through the C ABI. Default workload: the Wan-1.3B
 480p-shaped layer (B=1, H=12, N=32760, d=128, rho=0.1, nu=0.45).
 
-Prints one JSON line on rank 0. Multi-GPU (torchrun): every rank runs an independent
-replica of the workload (the path has no exchange step); the step time is the max over
-ranks and `value` counts the work of all ranks.
+Prints one JSON line on rank 0. Multi-GPU (torchrun): rank r runs batch element r of an
+N-element job, the workload's shape with its own seeded input (the path has no exchange
+step); the step time is the max over ranks and `value` counts the work of all ranks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 480p|720p|480p_14b|480p_topk015|dense|tiny]
   python bench.py --impl reference ...   # the CPU oracle on a bounded sample (rank 0)
@@ -177,7 +177,7 @@ def workload_config(wl):
             "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "grid_thw": list(wl.grid),
             "rho": wl.rho, "nu": wl.nu, "block": 64, "seed": wl.seeds[0],
             "l2": "no flush; per-step working set ~1.2 GB (inputs 300 MB + states) exceeds the 126 MB L2",
-            "parallelism": "replicas (no data-path collective)"}
+            "parallelism": "batch sharded over ranks: rank r runs element r (seed + r); no data-path collective"}
 
 
 # ------------------------------------------------------------------ clocks
@@ -229,9 +229,9 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ ranks
-# One process per GPU (torchrun). The path has no exchange step: every rank runs an
-# independent replica of the workload; ranks meet only for barriers around the timed
-# region and for the max of the per-rank times.
+# One process per GPU (torchrun). The path has no exchange step: rank r runs batch element
+# r of the job on its own; ranks meet only for barriers around the timed region and for
+# the max of the per-rank times.
 def rank_env():
     """(rank, world, local_rank) from the torchrun environment (1 process without it)."""
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
@@ -305,7 +305,8 @@ def run_ours(args, wl):
         return max_over_ranks_of(x, world, dev)
 
     S.lib()
-    q, k, v = make_workload_qkv(wl)
+    # rank r takes batch element r of an N-element job: its own seeded input, same shape
+    q, k, v = make_workload_qkv(wl, seed=wl.seeds[0] + rank)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     eng = S.SageSLA(wl.B, wl.H, wl.N, wl.rho, wl.nu, device=dev)
     stream = torch.cuda.current_stream(dev)

@@ -1,6 +1,6 @@
 """Multi-rank host logic of bench.py on CPU: two gloo ranks as spawned processes.
 
-The SageSLA path has no exchange step, so N GPUs run N independent replicas. What must
+The SageSLA path has no exchange step, so N GPUs run N batch elements independently. What must
 hold across ranks: every rank takes the same collective steps, the job's step time is the
 slowest rank's, the reported value counts the work of all ranks, and only rank 0 prints.
 """
