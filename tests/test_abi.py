@@ -97,6 +97,38 @@ def test_validation_rejects_before_launch(L):
                              p, p, 8, p, p, p, p, 16, None) == 1
 
 
+def test_more_validation_paths(L):
+    # every case below fails host-side checks, so no CUDA call is made
+    sh = _sh()
+    p = ctypes.c_void_p(0x1000)   # aligned, never dereferenced
+    mis = ctypes.c_void_p(0x1008)  # 8-byte aligned only
+    big = 1 << 40
+    # prepare: softmax scale must be positive and finite; the workspace must be large enough
+    for bad_scale in (0.0, -0.1, float("nan"), float("inf")):
+        assert L.sagesla_prepare(ctypes.byref(sh), p, p, p, bad_scale, *([p] * 9), p, big, None) == 1
+    assert L.sagesla_prepare(ctypes.byref(sh), p, p, p, 0.088, *([p] * 9), p, 64, None) == 1
+    # select: ratios, the marginal list when m > 0, the optional logits buffer
+    assert L.sagesla_select(ctypes.byref(sh), p, p, 1.5, 0.1, p, p, p, None, None) == 1
+    assert L.sagesla_select(ctypes.byref(sh), p, p, 0.25, 0.25, p, None, p, None, None) == 1
+    assert L.sagesla_select(ctypes.byref(sh), p, p, 0.25, 0.25, p, p, p, mis, None) == 1
+    assert L.sagesla_select(ctypes.byref(sh), p, p, 0.25, 0.25, p, mis, p, None, None) == 1
+    # the status word needs an aligned workspace of at least 256 bytes
+    assert L.sagesla_reset_status(None, 1 << 20, None) == 1
+    assert L.sagesla_reset_status(p, 128, None) == 1
+    assert L.sagesla_reset_status(mis, 1 << 20, None) == 1
+    # the no-workspace prepare: shape, pointers, scale, and the size of its fixed scratch
+    args = [p] * 3 + [ctypes.c_float(0.088)] + [p] * 9 + [None]
+    assert L.sagesla_prepare_static_scratch(None, *args) == 1
+    assert L.sagesla_prepare_static_scratch(ctypes.byref(_sh(d=64)), *args) == 2
+    assert L.sagesla_prepare_static_scratch(ctypes.byref(_sh(N=0)), *args) == 1
+    assert L.sagesla_prepare_static_scratch(ctypes.byref(sh), *([mis] * 3), ctypes.c_float(0.088),
+                                            *([p] * 9), None) == 1
+    assert L.sagesla_prepare_static_scratch(ctypes.byref(sh), *([p] * 3), ctypes.c_float(float("nan")),
+                                            *([p] * 9), None) == 1
+    # 64 heads of 8192 blocks need 256 MiB of block sums: more than the fixed 24 MiB
+    assert L.sagesla_prepare_static_scratch(ctypes.byref(_sh(H=64, N=8192 * 64)), *args) == 2
+
+
 def test_status_strings(L):
     for code, word in [(0, b"ok"), (1, b"invalid"), (2, b"unsupported"), (3, b"CUDA"), (4, b"timed out")]:
         assert word in L.sagesla_status_string(code)
