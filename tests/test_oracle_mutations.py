@@ -102,3 +102,55 @@ def test_mutation_rint_truncates(monkeypatch):
         assert _fails(pins.test_quantize_round_half_even_closed_form)
     finally:
         monkeypatch.undo()
+
+
+def test_mutation_scale_over_128(monkeypatch):
+    orig = S.quantize_blocks
+
+    def over_128(X, N, b=S.BLOCK):
+        x8, s = orig(X, N, b)
+        s128 = (s * np.float32(127) / np.float32(128)).astype(np.float32)
+        return x8, s128
+
+    monkeypatch.setattr(S, "quantize_blocks", over_128)
+    monkeypatch.setattr(pins.O, "quantize_blocks", over_128)
+    assert _fails(pins.test_quantize_round_half_even_closed_form)
+
+
+def test_mutation_softmax_scale_folded_twice(monkeypatch):
+    orig = S.prepare
+
+    def twice(q, k, v=None, c_s=None, b=S.BLOCK, smooth=True, exact=False):
+        cs = S.softmax_scale(np.asarray(q).shape[-1]) if c_s is None else c_s
+        return orig(np.asarray(q) * float(cs), k, v, c_s, b, smooth, exact)
+
+    monkeypatch.setattr(S, "prepare", twice)
+    assert _fails(lambda: pins.test_dense_unquantized_equals_sdpa(64))
+
+
+def test_mutation_linear_branch_on_unsmoothed_keys(monkeypatch):
+    orig = S.prepare
+
+    def unsmoothed(q, k, v=None, c_s=None, b=S.BLOCK, smooth=True, exact=False):
+        p = orig(q, k, v, c_s, b, smooth, exact)
+        p.k_t = np.asarray(k, dtype=p.k_t.dtype)  # phi(K) instead of phi(K~) downstream
+        return p
+
+    monkeypatch.setattr(S, "prepare", unsmoothed)
+    assert _fails(pins.test_k_shift_invariance_bitexact_full_method)
+
+
+def test_mutation_negligible_ties_to_lower_index(monkeypatch):
+    orig = S.select
+
+    def low_negligible(q_bar, k_bar, rho, nu):
+        sel = orig(q_bar, k_bar, rho, nu)
+        ell = sel.logits
+        nK = ell.shape[-1]
+        jj = np.broadcast_to(np.arange(nK), ell.shape)
+        low_first = np.lexsort((jj, ell.astype(np.float64)), axis=-1)  # lowest logit, lower index
+        neg = np.sort(low_first[..., :sel.n_neg], axis=-1).astype(np.int32)
+        return S.Selection(sel.k_c, sel.n_neg, sel.m, ell, sel.rank, sel.crit, sel.marg, neg)
+
+    monkeypatch.setattr(pins.O, "select", low_negligible)
+    assert _fails(pins.test_select_ties_go_to_lower_index)
