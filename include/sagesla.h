@@ -105,11 +105,19 @@ int sagesla_prepare(const sagesla_shape* shape, const void* q, const void* k,
  * before any launch. The first call on a device looks up the array's address with
  * cudaGetSymbolAddress and should come before any stream capture. All calls share the
  * array: calls whose kernels overlap on the GPU race on it (order them on one stream).
- * Nothing is allocated; a timed-out device wait is not reported by this variant. */
+ * Nothing is allocated. A timed-out device wait is recorded in the array's status word:
+ * read it with sagesla_static_scratch_status. */
 int sagesla_prepare_static_scratch(const sagesla_shape* shape, const void* q, const void* k,
                                    const void* v, float sm_scale, int8_t* q8, int8_t* k8,
                                    float* q_scale, float* k_scale, float* k_mean, float* q_bar,
                                    float* k_bar, void* h, float* z, void* stream);
+
+/* The status word of sagesla_prepare_static_scratch's internal array, for the current
+ * device: synchronizes `stream`, then returns SAGESLA_OK, SAGESLA_ERR_TIMEOUT if a bounded
+ * device wait of a static-scratch call gave up since that call began (its outputs are
+ * invalid), or SAGESLA_ERR_CUDA if the stream reported an error. Each static-scratch call
+ * clears the word when it starts. No counterpart in the paper (interface variant). */
+int sagesla_static_scratch_status(void* stream);
 
 /* Step (4): block logits, ranking and the per-row block lists.
  * Inputs : q_bar, k_bar fp32 [B,H,nB,d]; rho, nu as in sagesla_counts.
@@ -146,6 +154,43 @@ int sagesla_forward(const sagesla_shape* shape, const void* q, float sm_scale,
  * SAGESLA_ERR_TIMEOUT if a bounded device wait gave up (the affected output is
  * invalid), or SAGESLA_ERR_CUDA if the stream reported an error. */
 int sagesla_check_status(const void* workspace, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * W8A8 block-wise INT8 linear layer ("TurboDiffusion Demystified", section "Pillar Three:
+ * W8A8 Linear Layer Quantization": weights and activations of the linear layers in INT8,
+ * block-wise at 128x128 granularity). Y = X W^T + bias with X [M, K] and W [N, K] each
+ * cut into 128x128 tiles (rows x input channels; edge tiles ragged).
+ * ---------------------------------------------------------------------------------- */
+
+/* Quantize a bf16 matrix x [rows, K] (row-major) per 128x128 tile: s = fl32(amax/127),
+ * x8 = clamp(rint(fl32(x/s)), -127, 127) with ties to even (s = 0 and codes 0 for an
+ * all-zero tile). Outputs: x8 int8 [rows, K]; scale fp32 [ceil(rows/128), ceil(K/128)].
+ * Serves activations and weights alike. Requires K a multiple of 16 and ceil(rows/128) <=
+ * 65535; x and x8 16-byte aligned. The codes and the scales' bits are deterministic. */
+int sagesla_w8a8_quantize(const void* x, int rows, int K, int8_t* x8, float* scale,
+                          void* stream);
+
+/* Y bf16 [M, N] = sum_kb sx[m/128, kb] * sw[n/128, kb] * (x8[m, kb-tile] . w8[n, kb-tile])
+ * + bias[n], from the outputs of sagesla_w8a8_quantize for X (x8, sx) and W (w8, sw).
+ * bias: fp32 [N] or NULL. Each K tile's exact integer partial sum is scaled in fp32 (the
+ * scale product rounded to fp32) into an fp32 accumulator; the sum is rounded once to
+ * bf16. Requires K a multiple of 16 (<= 16384) and N a multiple of 8; x8, w8, y and
+ * workspace 16-byte aligned. workspace: >= 256 bytes; its status word records a timed-out
+ * device wait (read it with sagesla_check_status). */
+int sagesla_w8a8_linear(const int8_t* x8, const float* sx, const int8_t* w8, const float* sw,
+                        const float* bias, void* y, int M, int N, int K, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* Diagnostics for the failure path (no counterpart in the paper). Launches one small
+ * kernel that waits on an mbarrier nothing ever arrives on, through the same bounded wait
+ * every kernel of this library uses, with a limit of limit_us microseconds (1..1000000).
+ * The wait runs out, the kernel ORs the timeout bit into the workspace status word and
+ * returns; the next sagesla_check_status returns SAGESLA_ERR_TIMEOUT and the CUDA context
+ * stays usable (clear the word with sagesla_reset_status). workspace: >= 256 bytes, 16-byte
+ * aligned. Returns SAGESLA_ERR_INVALID_ARG for a bad pointer or limit, SAGESLA_ERR_CUDA if
+ * the launch failed. */
+int sagesla_selftest_wait_timeout(void* workspace, size_t workspace_bytes,
+                                  unsigned int limit_us, void* stream);
 
 /* Launch tracing (diagnostics). While enabled, every kernel launch made by this library
  * is bracketed by a pair of CUDA events recorded on its launch stream. Process-global

@@ -21,8 +21,9 @@
 //     word is cleared (cudaMemsetAsync, no allocation) at the start of every call. Calls
 //     whose kernels overlap on the GPU (different streams, no ordering between them) race
 //     on the array and give wrong results: order them on one stream.
-//   * A bounded device wait that gives up is recorded in the array's status word, which
-//     callers cannot read; the outputs of such a call are invalid.
+//   * A bounded device wait that gives up is recorded in the array's status word; read it
+//     with sagesla_static_scratch_status (which synchronizes the stream). The outputs of
+//     such a call are invalid.
 #include <mutex>
 
 #include "../../include/sagesla.h"
@@ -97,4 +98,16 @@ extern "C" int sagesla_prepare_static_scratch(const sagesla_shape* shape, const 
                                             k_mean, q_bar, k_bar, h, z,
                                             static_cast<char*>(scratch), st);
   return e == cudaSuccess ? SAGESLA_OK : SAGESLA_ERR_CUDA;
+}
+
+extern "C" int sagesla_static_scratch_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SAGESLA_ERR_CUDA;
+  void* scratch = nullptr;
+  if (sgs::scratch_address(&scratch) != cudaSuccess) return SAGESLA_ERR_CUDA;
+  int word = 0;  // the status word sits at offset 0 of the array (workspace layout)
+  if (cudaMemcpy(&word, scratch, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SAGESLA_ERR_CUDA;
+  if (word & sgs::kStatusTimeoutBit) return SAGESLA_ERR_TIMEOUT;
+  return word ? SAGESLA_ERR_CUDA : SAGESLA_OK;
 }

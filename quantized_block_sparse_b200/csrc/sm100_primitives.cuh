@@ -83,22 +83,29 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t par
 }
 
 // Wait for the phase with the given parity to complete. Gives up (returns false) when
-// another thread of the CTA has raised *abort, or after kWaitLimitNs; on a timeout it
-// raises *abort and ORs kStatusTimeout into *status so the host can see it. Between checks
-// the thread is suspended in try_wait (hint 1 ms), so waiting costs few instructions.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          int* status) {
+// another thread of the CTA has raised *abort, or after limit_ns; on a timeout it raises
+// *abort and ORs kStatusTimeout into *status so the host can see it. Between checks the
+// thread is suspended in try_wait (hint 1 ms, or the limit if shorter), so waiting costs
+// few instructions.
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity,
+                                                volatile int* abort, int* status,
+                                                unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t hint = limit_ns < 1000000ull ? static_cast<uint32_t>(limit_ns) : 1000000u;
   const unsigned long long t0 = globaltimer();
   for (;;) {
-    if (mbar_try_wait_suspend(bar, parity, 1000000u)) return true;
+    if (mbar_try_wait_suspend(bar, parity, hint)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
       if (status) atomicOr(status, kStatusTimeout);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          int* status) {
+  return mbar_wait_limit(bar, parity, abort, status, kWaitLimitNs);
 }
 
 // After an aborted wait: wait (again bounded, ignoring the abort flag) for copies or MMAs

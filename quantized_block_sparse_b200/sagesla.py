@@ -56,6 +56,15 @@ def lib():
     L.sagesla_prepare.restype = ctypes.c_int
     L.sagesla_prepare_static_scratch.argtypes = [sp, _vp, _vp, _vp, ctypes.c_float] + [_vp] * 9 + [_vp]
     L.sagesla_prepare_static_scratch.restype = ctypes.c_int
+    L.sagesla_static_scratch_status.argtypes = [_vp]
+    L.sagesla_static_scratch_status.restype = ctypes.c_int
+    L.sagesla_selftest_wait_timeout.argtypes = [_vp, ctypes.c_size_t, ctypes.c_uint, _vp]
+    L.sagesla_selftest_wait_timeout.restype = ctypes.c_int
+    L.sagesla_w8a8_quantize.argtypes = [_vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp]
+    L.sagesla_w8a8_quantize.restype = ctypes.c_int
+    L.sagesla_w8a8_linear.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+    L.sagesla_w8a8_linear.restype = ctypes.c_int
     L.sagesla_select.argtypes = [sp, _vp, _vp, ctypes.c_double, ctypes.c_double, _vp, _vp, _vp, _vp, _vp]
     L.sagesla_select.restype = ctypes.c_int
     L.sagesla_forward.argtypes = ([sp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int,
@@ -188,6 +197,11 @@ def sagesla_prepare_static_scratch(q, k, v, sm_scale=None, out: Prepared | None 
     return out
 
 
+def sagesla_static_scratch_status(stream=None):
+    """Raise if a bounded device wait of a static-scratch prepare gave up (synchronizes)."""
+    _check(lib().sagesla_static_scratch_status(_stream(stream)), "static scratch status")
+
+
 def alloc_selection(B, H, N, rho, nu, device="cuda", logits=False) -> Selection:
     nB, k_c, n_neg, m = sagesla_counts(B, H, N, rho, nu)
     nBp = -(-nB // 64) * 64
@@ -230,6 +244,13 @@ def sagesla_check_status(workspace, stream=None):
     _check(lib().sagesla_check_status(_ptr(workspace), _stream(stream)), "device status")
 
 
+def sagesla_selftest_wait_timeout(workspace, limit_us: int, stream=None):
+    """Diagnostics: run a kernel whose bounded wait must run out after limit_us (the
+    failure path of every kernel); sagesla_check_status then reports the timeout."""
+    _check(lib().sagesla_selftest_wait_timeout(_ptr(workspace), workspace.numel(), int(limit_us),
+                                                _stream(stream)), "sagesla_selftest_wait_timeout")
+
+
 class SageSLA:
     """All three calls for one shape, with buffers allocated once (device memory via torch)."""
 
@@ -251,3 +272,28 @@ class SageSLA:
 
     def check(self, stream=None):
         sagesla_check_status(self.workspace, stream)
+
+
+# ---------------------------------------------------------------- W8A8 linear layer
+def sagesla_w8a8_quantize(x, stream=None):
+    """bf16 [rows, K] -> (int8 codes [rows, K], fp32 scales [ceil(rows/128), ceil(K/128)])."""
+    assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and x.dim() == 2
+    R, K = x.shape
+    x8 = torch.empty(R, K, dtype=torch.int8, device=x.device)
+    s = torch.empty(-(-R // 128), -(-K // 128), dtype=torch.float32, device=x.device)
+    _check(lib().sagesla_w8a8_quantize(_ptr(x), R, K, _ptr(x8), _ptr(s), _stream(stream)),
+           "sagesla_w8a8_quantize")
+    return x8, s
+
+
+def sagesla_w8a8_linear(x8, sx, w8, sw, bias=None, workspace=None, out=None, stream=None):
+    """Y bf16 [M, N] = X W^T + bias from the quantized operands."""
+    M, K = x8.shape
+    N = w8.shape[0]
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=x8.device)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=x8.device) if out is None else out
+    _check(lib().sagesla_w8a8_linear(_ptr(x8), _ptr(sx), _ptr(w8), _ptr(sw), _ptr(bias), _ptr(y),
+                                     M, N, K, _ptr(workspace), workspace.numel(), _stream(stream)),
+           "sagesla_w8a8_linear")
+    return y

@@ -127,6 +127,12 @@ def test_more_validation_paths(L):
                                             *([p] * 9), None) == 1
     # 64 heads of 8192 blocks need 256 MiB of block sums: more than the fixed 24 MiB
     assert L.sagesla_prepare_static_scratch(ctypes.byref(_sh(H=64, N=8192 * 64)), *args) == 2
+    # the failure-path self-test: workspace pointer and size, limit in 1..10^6 microseconds
+    assert L.sagesla_selftest_wait_timeout(None, 1 << 20, 1000, None) == 1
+    assert L.sagesla_selftest_wait_timeout(mis, 1 << 20, 1000, None) == 1
+    assert L.sagesla_selftest_wait_timeout(p, 128, 1000, None) == 1
+    assert L.sagesla_selftest_wait_timeout(p, 1 << 20, 0, None) == 1
+    assert L.sagesla_selftest_wait_timeout(p, 1 << 20, 1000001, None) == 1
 
 
 def test_status_strings(L):
