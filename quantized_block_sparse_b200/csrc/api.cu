@@ -27,7 +27,7 @@ WsLayout ws_layout(const Dims& g) {
   L.Zbuf = off;
   off = align256(off + static_cast<size_t>(g.BH) * g.nB * kHeadDim * 4);
   L.Zb = off;
-  off = align256(off + static_cast<size_t>(g.BH) * g.nB * kHeadDim * 2);
+  off = align256(off + static_cast<size_t>(g.BH) * g.nB * kHeadDim * 2 * 2);
   L.pairs = off;
   off = align256(off + static_cast<size_t>(g.BH) * g.nB * 8);
   L.pair_counts = off;

@@ -11,9 +11,11 @@
 //   hgemm_kernel   H = M . h per head, M the 0/1 marginal mask [nB x nBp] and h viewed as
 //                  [nB x d*d]: a persistent tcgen05 bf16 GEMM (fp32 accumulation in two
 //                  TMEM accumulators), 128x256 output tiles, TMA-fed 4-stage pipeline,
-//                  bf16 output; plus one 128-column tile for Z.
-//   zb_kernel      z_j rounded to bf16; hgemm_kernel's extra column tile gives Z = M . z
-//                  (bf16 operands, fp32 accumulation and output, like H).
+//                  bf16 output; plus one 256-column tile for Z.
+//   zb_kernel      z_j split into two bf16 parts, z_hi = bf16(z) and z_lo = bf16(z - z_hi);
+//                  hgemm_kernel's extra column tile multiplies M by [z_hi | z_lo] (exact
+//                  0/1 x bf16 products, fp32 accumulation) and Z = M.z_hi + M.z_lo in fp32,
+//                  so Z keeps about 17 significant bits of z instead of bf16's 8.
 //   linout_kernel  per pair of adjacent query blocks: phi(Q~) (recomputed from Q, bf16)
 //                  times H_i on tcgen05 (M = 128 rows = both blocks, one MMA chain per
 //                  block), divided by phi(Q~) . Z_i; bf16 O_l for the attention epilogue.
@@ -29,8 +31,8 @@ namespace {
 // tiles halve the mask re-reads, the main L2 traffic). Warp 0 streams A/B k-blocks through
 // a 4-stage ring with TMA, warp 1 issues the MMAs (M128 N256 K16) into one of two 256-column
 // TMEM accumulators, warps 2-5 drain the other accumulator (bf16) while the next tile runs.
-// One more, 128-column tile per row block computes Z = M . z from z rounded to bf16 (the
-// same operand precision as h) and is written in fp32.
+// One more 256-column tile per row block computes M . [z_hi | z_lo] (z split into two bf16
+// parts by zb_kernel); its drain adds the two halves and writes Z in fp32.
 constexpr int kGemmStages = 4;
 constexpr int kGemmStageBytes = 16384 + 32768;
 constexpr int kGemmThreads = 192;
@@ -94,15 +96,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_con
           }
           const uint32_t sa = smem_u32(smem + s * kGemmStageBytes);
           const uint32_t sb = sa + 16384;
-          mbar_expect_tx(smem_u32(full + s), nt < kNTH ? kGemmStageBytes : 16384 + 16384);
+          mbar_expect_tx(smem_u32(full + s), kGemmStageBytes);
           tma_load_3d(sa, &tmA, smem_u32(full + s), kb * 64, mt * 128, bh);
           if (nt < kNTH) {
 #pragma unroll
             for (int g = 0; g < 4; ++g)
               tma_load_3d(sb + 8192 * g, &tmB, smem_u32(full + s), nt * 256 + 64 * g, kb * 64, bh);
           } else {
-            tma_load_3d(sb, &tmZ, smem_u32(full + s), 0, kb * 64, bh);
-            tma_load_3d(sb + 8192, &tmZ, smem_u32(full + s), 64, kb * 64, bh);
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+              tma_load_3d(sb + 8192 * g, &tmZ, smem_u32(full + s), 64 * g, kb * 64, bh);
           }
         }
       }
@@ -112,8 +115,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_con
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc_h = make_idesc(1, 1, 0, 1, 128, 256);
-      constexpr uint32_t idesc_z = make_idesc(1, 1, 0, 1, 128, 128);
+      constexpr uint32_t idesc = make_idesc(1, 1, 0, 1, 128, 256);
       int it = 0, lt = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++lt) {
@@ -123,7 +125,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_con
           break;
         }
         tc_fence_after();
-        const uint32_t idesc = (tile % kNT) < kNTH ? idesc_h : idesc_z;
         for (int kb = 0; kb < nK; ++kb, ++it) {
           const int s = it % kGemmStages;
           if (!mbar_wait(smem_u32(full + s), (it / kGemmStages) & 1, &abort_flag, status)) {
@@ -172,15 +173,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_con
           }
         }
       } else {
+        // columns [0,128): M . z_hi, [128,256): M . z_lo; Z = their fp32 sum
         float* dst = Zout + (static_cast<size_t>(bh) * nB + i) * kHeadDim;
 #pragma unroll
         for (int cchunk = 0; cchunk < 4; ++cchunk) {
-          uint32_t r[32];
-          tmem_ld32_sync(taddr + (static_cast<uint32_t>(32 * wq) << 16) + 256 * a + 32 * cchunk, r);
+          uint32_t rh[32], rl[32];
+          const uint32_t ta = taddr + (static_cast<uint32_t>(32 * wq) << 16) + 256 * a + 32 * cchunk;
+          tmem_ld32_sync(ta, rh);
+          tmem_ld32_sync(ta + 128, rl);
           if (i < nB) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cchunk);
+            float4* d4 = reinterpret_cast<float4*>(dst + 32 * cchunk);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) d4[q] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+            for (int q = 0; q < 8; ++q) {
+              float f[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                f[e] = __fadd_rn(__uint_as_float(rh[4 * q + e]), __uint_as_float(rl[4 * q + e]));
+              d4[q] = make_float4(f[0], f[1], f[2], f[3]);
+            }
           }
         }
       }
@@ -193,14 +203,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) hgemm_kernel(const __grid_con
   if (warp == 1) tmem_dealloc(taddr, 512);
 }
 
-// ------------------------------------------------------------------ z -> bf16
-// z_j rounded to bf16 (RNE): the B operand of the Z column tile of hgemm_kernel.
+// ------------------------------------------------------------------ z -> bf16 hi + lo
+// The B operand of the Z column tile of hgemm_kernel: row j of zb is [z_hi | z_lo] (2 x 128
+// bf16), z_hi = bf16(z_j) and z_lo = bf16(z_j - z_hi) (the subtraction is exact), both RNE.
+// x indexes groups of 4 channels: row j = x / 32, channels 4*(x % 32) .. +3.
+__device__ __forceinline__ float bf16_round(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
 __global__ void __launch_bounds__(256) zb_kernel(const float4* __restrict__ z,
                                                  uint2* __restrict__ zb, size_t n4) {
   for (size_t x = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; x < n4;
        x += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const float4 v = z[x];
-    zb[x] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+    const float4 h = make_float4(bf16_round(v.x), bf16_round(v.y), bf16_round(v.z), bf16_round(v.w));
+    const size_t row = x >> 5, c4 = x & 31;
+    zb[row * 64 + c4] = make_uint2(pack_bf16x2(h.x, h.y), pack_bf16x2(h.z, h.w));
+    zb[row * 64 + 32 + c4] = make_uint2(pack_bf16x2(v.x - h.x, v.y - h.y), pack_bf16x2(v.z - h.z, v.w - h.w));
   }
 }
 
@@ -368,7 +386,7 @@ cudaError_t launch_linear(const Dims& g, const void* q, float sm_scale, const vo
   if (!make_tmap_3d(&tmA, mask, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.nBp, g.nB, g.BH, 64, 128) ||
       !make_tmap_3d(&tmB, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim * kHeadDim, g.nB, g.BH, 64,
                     64) ||
-      !make_tmap_3d(&tmZ, Zb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim, g.nB, g.BH, 64, 64) ||
+      !make_tmap_3d(&tmZ, Zb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 2 * kHeadDim, g.nB, g.BH, 64, 64) ||
       !make_tmap_3d(&tmH, Hbuf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim,
                     static_cast<uint64_t>(g.nB) * kHeadDim, g.BH, 64, 128) ||
       !make_tmap_3d(&tmQ, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim, g.N, g.BH, 64, 64) ||

@@ -26,7 +26,7 @@ struct WsLayout {
   size_t mu_part;    // fp32 [BH, nB, d]   per-block channel sums of K
   size_t Hbuf;       // bf16 [BH, nB, d, d]
   size_t Zbuf;       // fp32 [BH, nB, d]
-  size_t Zb;         // bf16 [BH, nB, d]      z rounded to bf16 (the Z GEMM operand)
+  size_t Zb;         // bf16 [BH, nB, 2d]     [z_hi | z_lo], z split into two bf16 parts
   size_t pairs;      // int2 [BH, nB]         query-block pairs of the attention tiles
   size_t pair_counts;  // int32 [BH, ceil(nB/64)] tiles per pairing segment
   size_t Ol;         // bf16 [BH, N, d]
