@@ -52,8 +52,18 @@ class Workload:
 
 # Workloads for parity and measurement. Shapes follow the Wan latent grids (480p:
 # 21x30x52 tokens, 720p: 21x45x80) with head dim 128: the 1.3B model has 12 heads, the
-# 14B models 40. "480p_14b" (Wan2.1-14B at 480p) and "480p_topk015" (--sla_topk 0.15 on
-# the 1.3B layer) are second workloads on the same kernels.
+# 14B models 40. Second workloads on the same kernels: "480p_14b" (Wan2.1-14B at 480p),
+# "480p_topk015" (--sla_topk 0.15 on the 1.3B layer) and "720p_i2v" (Wan2.2-I2V-A14B at
+# 720p: its DiT sees the same 21x45x80 token grid and 40 heads as the 14B T2V layer, the
+# image condition entering through the input channels, so only the seed differs).
+SWEEP_RHOS = (1.0, 0.5, 0.2, 0.1, 0.05)
+
+
+def sweep_workload(rho: float) -> Workload:
+    """480p-shaped sweep point: B=2, nu=(1-rho)/2, seeds 0 and 1."""
+    return Workload(f"sweep_rho{rho:g}", 2, 12, (21, 30, 52), rho, (1.0 - rho) / 2.0, (0, 1))
+
+
 WORKLOADS = {
     "tiny": Workload("tiny", 1, 2, (4, 16, 16), 0.25, 0.25),
     "dense": Workload("dense", 1, 12, (4, 32, 32), 1.0, 0.0),
@@ -61,13 +71,9 @@ WORKLOADS = {
     "720p": Workload("720p", 1, 40, (21, 45, 80), 0.10, 0.45),
     "480p_14b": Workload("480p_14b", 1, 40, (21, 30, 52), 0.10, 0.45),
     "480p_topk015": Workload("480p_topk015", 1, 12, (21, 30, 52), 0.15, 0.45),
+    "720p_i2v": Workload("720p_i2v", 1, 40, (21, 45, 80), 0.10, 0.45, (1,)),
 }
-SWEEP_RHOS = (1.0, 0.5, 0.2, 0.1, 0.05)
-
-
-def sweep_workload(rho: float) -> Workload:
-    """480p-shaped sweep point: B=2, nu=(1-rho)/2, seeds 0 and 1."""
-    return Workload(f"sweep_rho{rho:g}", 2, 12, (21, 30, 52), rho, (1.0 - rho) / 2.0, (0, 1))
+WORKLOADS.update({f"sweep_rho{r:g}": sweep_workload(r) for r in SWEEP_RHOS})
 
 
 def _head_fields(rng: np.random.Generator, grid, d: int):

@@ -56,6 +56,12 @@ def test_dense_workload_sageattention_only():
 
 
 @pytest.mark.parametrize("N,rho,nu", [
+    (1, 1.0, 0.0),       # one token: a single block with 63 padded rows and keys
+    (17, 0.5, 0.2),      # one ragged block smaller than a tile (nB = 1, so k_c = 1, m = 0)
+    (40, 1.0, 0.0),
+    (63, 0.3, 0.3),
+    (130, 0.34, 0.33),   # three blocks, the last of 2 tokens: k_c = 2, n_neg = 0, m = 1
+    (150, 0.25, 0.3),    # three blocks: k_c = 1, m = 2 (linear branch on a ragged tail)
     (64, 1.0, 0.0),      # a single block
     (65, 0.5, 0.0),      # two blocks, the second holds one token
     (100, 0.5, 0.5),     # ragged, no marginal blocks (m = 0), one negligible
@@ -129,6 +135,23 @@ def test_480p_full_size_sampled():
 
 def test_720p_full_size_sampled():
     near, res = _sampled_check(WORKLOADS["720p"], heads_for_oracle=2, qblocks_per_head=12)
+    assert near == 0
+
+
+def test_480p_topk015_full_size_sampled():
+    # --sla_topk 0.15: k_c = 77 critical blocks per row (odd), m = 205
+    near, res = _sampled_check(WORKLOADS["480p_topk015"], heads_for_oracle=2, qblocks_per_head=12)
+    assert near == 0
+
+
+def test_480p_14b_full_size_sampled():
+    # Wan2.1-14B at 480p: 40 heads; heads 0-1 compared against the oracle
+    near, res = _sampled_check(WORKLOADS["480p_14b"], heads_for_oracle=2, qblocks_per_head=8)
+    assert near == 0
+
+
+def test_720p_i2v_full_size_sampled():
+    near, res = _sampled_check(WORKLOADS["720p_i2v"], heads_for_oracle=1, qblocks_per_head=8, seed=1)
     assert near == 0
 
 
