@@ -9,7 +9,7 @@ Prints one JSON line on rank 0. Multi-GPU (torchrun): rank r runs batch element 
 N-element job, the workload's shape with its own seeded input (the path has no exchange
 step); the step time is the max over ranks and `value` counts the work of all ranks.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 480p|720p|480p_14b|480p_topk015|dense|tiny]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME|sweep]
   python bench.py --impl reference ...   # the CPU oracle on a bounded sample (rank 0)
 """
 from __future__ import annotations
@@ -28,17 +28,30 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from quantized_block_sparse_b200.inputs import WORKLOADS, make_workload_qkv  # noqa: E402
+from quantized_block_sparse_b200.inputs import SWEEP_RHOS, WORKLOADS, make_workload_qkv  # noqa: E402
 
 METRIC = "SageSLA fwd ms/call & dense-equiv TOPS at Wan-1.3B 480p shape; % tensor roofline"
 UNIT = "dense-equiv TOPS"
 INT8_TO_BF16_RATE = 2.0  # dense INT8 : BF16 tensor rate on B200: nominal 4.5 : 2.25 POPS;
                          # a tcgen05 M128 N128 issue-rate probe gave 8124 : 4064 MAC/clk/SM
+PROBE_BF16_MAC_PER_CLK_SM = 4064  # that probe's bf16 rate: back-to-back kind::f16 MMAs
+N_SM = 148
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
 def dense_equiv_ops(wl) -> float:
     return 4.0 * wl.B * wl.H * float(wl.N) ** 2 * wl.d
+
+
+def forward_work(wl, nB, k_c, m):
+    """Algorithmic tensor work of one sagesla_forward over the executed blocks: INT8 QK^T
+    ops and BF16 flops (P.V over the critical pairs, the marginal gather-sum and the
+    phi(Q~).H product per query block)."""
+    heads = wl.B * wl.H
+    pair = 2.0 * 64 * 64 * 128
+    int8 = heads * nB * k_c * pair
+    bf16 = heads * nB * (k_c * pair + (2.0 * m * 128 * 129 + 2.0 * 64 * 128 * 129 if m > 0 else 0.0))
+    return {"int8_ops": int8, "bf16_flops": bf16}
 
 
 def profiled_traffic(workload: str):
@@ -82,80 +95,86 @@ def load_peaks():
 
 
 # ------------------------------------------------------------------ CPU oracle timing
-def oracle_sample(q, k, v, wl, n_small=None, n_large=None):
-    """Time the CPU oracle on one head and scale to the whole call.
+def _oracle_rows(args):
+    """Worker: the oracle's forward (steps 5-7) for some query blocks of one head."""
+    prep, v, sel, qblocks = args
+    from threadpoolctl import threadpool_limits
 
-    Default (the cpu_baseline leg): one whole head, prepare + select + forward over all
-    nB query blocks; call time = B*H * that (heads are independent and equal in work).
-    With n_small/n_large (the per-step sample of --impl reference): forward runs on two
-    block-set sizes and a linear fit a + b*|S| splits the per-head fixed part (linear
-    states, H = M h) from the per-block part; call time = B*H * (prep_sel + a + b*nB).
+    import oracle as O
+    with threadpool_limits(1):
+        O.forward(prep, v, sel, heads=[(0, 0)], qblocks=qblocks)
+    return len(qblocks)
+
+
+def _warm(_):
+    """Worker start-up task: keeps the worker busy briefly so every worker gets spawned."""
+    time.sleep(0.5)
+    return os.getpid()
+
+
+def oracle_pool(wl, procs=None):
+    """A spawn-started process pool for the oracle's forward, its workers already running."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    nB = -(-wl.N // 64)
+    procs = procs or max(1, min(len(os.sched_getaffinity(0)), nB, 32))
+    ex = cf.ProcessPoolExecutor(procs, mp_context=mp.get_context("spawn"))
+    list(ex.map(_warm, range(procs)))
+    return ex, procs
+
+
+def oracle_head_time(q, k, v, wl, pool):
+    """Time the CPU oracle on one whole head of the workload, as it stands.
+
+    prepare and select run in this process; the forward's query blocks are split into one
+    contiguous chunk per worker of `pool` (from oracle_pool: spawn-started, one BLAS thread
+    each). Every worker recomputes the head's linear states, as the oracle does per call.
+    Returns (seconds, processes used, sample text).
     """
     import oracle as O
-    from threadpoolctl import threadpool_info
-
-    qf = q[:1, :1].float().numpy()
-    kf = k[:1, :1].float().numpy()
-    vf = v[:1, :1].float().numpy()
+    ex, procs = pool
     nB = -(-wl.N // 64)
+    qf, kf, vf = (t[:1, :1].float().numpy() for t in (q, k, v))
+    chunks = [c.tolist() for c in np.array_split(np.arange(nB), procs) if len(c)]
     t0 = time.perf_counter()
     prep = O.prepare(qf, kf)
     sel = O.select(prep.q_bar, prep.k_bar, wl.rho, wl.nu)
-    t_ps = time.perf_counter() - t0
-    if n_small is None:
-        t1 = time.perf_counter()
-        O.forward(prep, vf, sel, heads=[(0, 0)])
-        t_fwd = time.perf_counter() - t1
-        per_head = t_ps + t_fwd
-        wall = per_head
-        sample = (f"1 of {wl.B * wl.H} heads, whole: prepare+select+forward over all {nB} query "
-                  f"blocks ({wall:.1f} s of CPU work); call time = B*H * per-head time")
-    else:
-        rng = np.random.default_rng(0)
-        ts = []
-        for n in (n_small, n_large):
-            blocks = sorted(rng.choice(nB, size=min(n, nB), replace=False).tolist())
-            t1 = time.perf_counter()
-            O.forward(prep, vf, sel, heads=[(0, 0)], qblocks=blocks)
-            ts.append((len(blocks), time.perf_counter() - t1))
-        (n1, t1), (n2, t2) = ts
-        b = max((t2 - t1) / max(n2 - n1, 1), 0.0)
-        a = max(t1 - b * n1, 0.0)
-        per_head = t_ps + a + b * nB
-        wall = t_ps + t1 + t2
-        sample = (f"1 of {wl.B * wl.H} heads: prepare+select, forward on {n1} and {n2} of {nB} "
-                  f"query blocks; call time extrapolated as B*H*(prep_sel + a + b*nB); "
-                  f"{wall:.1f} s of CPU work")
-    est_s = wl.B * wl.H * per_head
-    cores = 0
-    for info in threadpool_info():
-        cores = max(cores, int(info.get("num_threads", 0)))
-    cores = cores or os.cpu_count()
-    return est_s, cores, sample
+    done = sum(ex.map(_oracle_rows, [(prep, vf, sel, c) for c in chunks]))
+    secs = time.perf_counter() - t0
+    assert done == nB
+    sample = (f"1 of {wl.B * wl.H} heads, whole and measured: prepare+select in one process, "
+              f"forward over all {nB} query blocks split across {len(chunks)} spawned processes "
+              f"(each recomputes the head's linear states); {secs:.1f} s wall")
+    return secs, len(chunks), sample
 
 
 def run_reference(args, wl):
-    """`--impl reference`: the CPU oracle, as it stands, on a bounded sample per step."""
+    """`--impl reference`: the CPU oracle, as it stands, on one whole head per step."""
     rank, _, _ = rank_env()
     if rank != 0:
         return 0
     q, k, v = make_workload_qkv(wl)
-    ests = []
+    times = []
     cores, sample = 0, ""
-    for step in range(args.warmup + args.steps):
-        est_s, cores, sample = oracle_sample(q, k, v, wl, n_small=2, n_large=6)
-        if step >= args.warmup:
-            ests.append(est_s)
-    est = statistics.mean(ests)
-    value = dense_equiv_ops(wl) / est / 1e12
+    pool = oracle_pool(wl)
+    try:
+        for step in range(args.warmup + args.steps):
+            secs, cores, sample = oracle_head_time(q, k, v, wl, pool)
+            if step >= args.warmup:
+                times.append(secs)
+    finally:
+        pool[0].shutdown()
+    per_head = statistics.mean(times)
+    value = dense_equiv_ops(wl) / (wl.B * wl.H) / per_head / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": est * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": per_head * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64/f32 (CPU oracle)", "data": "synthetic",
         "config": workload_config(wl),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample + "; one step = one head (value = one head's "
+                                            "dense-equivalent ops / its measured time)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -167,9 +186,12 @@ WORKLOAD_TITLES = {
     "720p": "Wan-14B 720p-shaped SageSLA layer",
     "480p_14b": "Wan2.1-14B 480p-shaped SageSLA layer",
     "480p_topk015": "Wan-1.3B 480p-shaped SageSLA layer, sla_topk 0.15",
-    "dense": "dense SageSLA test layer (rho = 1)",
+    "720p_i2v": "Wan2.2-I2V-A14B 720p-shaped SageSLA layer",
+    "dense": "dense SageAttention layer (rho = 1, no linear branch)",
     "tiny": "tiny SageSLA test layer",
 }
+WORKLOAD_TITLES.update({f"sweep_rho{r:g}": f"480p sparsity sweep, B=2, rho={r:g}, nu=(1-rho)/2"
+                        for r in SWEEP_RHOS})
 
 
 def workload_config(wl):
@@ -425,6 +447,12 @@ def run_ours(args, wl):
     att_ms = kern.get("attn_kernel", {}).get("avg_ms", float("nan"))
     achieved = bf16_equiv / (att_ms * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
+    # second denominator: the tcgen05 probe rate at the SM clock sampled during the run
+    sm_mhz = clk.get("sm_mhz") or 1965.0
+    peak_probe = PROBE_BF16_MAC_PER_CLK_SM * 2 * N_SM * sm_mhz * 1e6 / 1e12
+    # forward-level roofline: every executed block of sagesla_forward on the tensor pipe
+    fwd = forward_work(wl, nB, k_c, m)
+    t_roof_s = fwd["int8_ops"] / (INT8_TO_BF16_RATE * peak * 1e12) + fwd["bf16_flops"] / (peak * 1e12)
 
     line = {
         "metric": METRIC,
@@ -442,10 +470,22 @@ def run_ours(args, wl):
                      "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak,
                      "traffic": profiled_traffic(wl.name),
+                     "peak_tcgen05_probe": peak_probe, "frac_tcgen05_probe": achieved / peak_probe,
                      "note": (f"bf16-equivalent: INT8 QK^T ops / {INT8_TO_BF16_RATE:g} + BF16 PV flops over "
-                              f"{pairs} executed 64x64 block pairs; peak = {peak_src} cuBLAS bf16 burst; "
-                              f"traffic = DRAM bytes per launch from the committed ncu summary "
-                              f"(null once the kernel source differs from the profiled one)")},
+                              f"{pairs} executed 64x64 block pairs; peak = {peak_src} cuBLAS bf16 burst "
+                              f"(of {peak_src}); peak_tcgen05_probe = {PROBE_BF16_MAC_PER_CLK_SM} bf16 "
+                              f"MAC/clk/SM x 2 x {N_SM} SMs x the sampled SM clock; traffic = DRAM bytes "
+                              f"per launch from the committed ncu summary (null once the kernel source "
+                              f"differs from the profiled one)")},
+        "roofline_forward": {"bound": "tensor", "int8_ops": fwd["int8_ops"],
+                             "bf16_flops": fwd["bf16_flops"], "t_roof_ms": t_roof_s * 1e3,
+                             "fwd_ms": fwd_ms, "frac": t_roof_s * 1e3 / fwd_ms if fwd_ms else None,
+                             "frac_tcgen05_probe": (t_roof_s * 1e3 * peak / peak_probe / fwd_ms
+                                                    if fwd_ms else None),
+                             "note": "sagesla_forward over the executed blocks: INT8 QK^T (critical "
+                                     "pairs) at 2x the bf16 peak; BF16 P.V, the marginal gather "
+                                     "2*m*128*129 and phi(Q)H 2*64*128*129 per query block (if m > 0) "
+                                     "at the bf16 peak; frac = t_roof / measured forward time"},
         "e2e": {"value": whole_job_tops(dense_equiv_ops(wl), world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "pinned_host_memory": "GPU-local NUMA node" if local_cpus else "default placement"},
@@ -453,13 +493,103 @@ def run_ours(args, wl):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        est_s, cores, sample = oracle_sample(q, k, v, wl)
-        line["cpu_baseline"] = {"value": dense_equiv_ops(wl) / est_s / 1e12, "unit": UNIT,
-                                "cores": cores, "kind": "oracle", "sample": sample,
-                                "ms_per_call_est": est_s * 1e3}
+        pool = oracle_pool(wl)
+        try:
+            secs, cores, sample = oracle_head_time(q, k, v, wl, pool)
+        finally:
+            pool[0].shutdown()
+        line["cpu_baseline"] = {"value": dense_equiv_ops(wl) / (wl.B * wl.H) / secs / 1e12,
+                                "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                                "ms_per_head": secs * 1e3}
     if rank == 0:
         print(json.dumps(line), flush=True)
     del eng
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_heads(args, wl):
+    """`--parallel heads`: one layer's B*H heads split over the ranks (strong scaling).
+
+    Rank r runs prepare -> select -> forward on its contiguous range of heads; with
+    --gather (the default) every step ends with an all-gather of the outputs, so each rank
+    holds the whole layer's output. value = the whole layer's dense-equivalent ops over the
+    slowest rank's step time.
+    """
+    import torch
+    import torch.distributed as dist
+
+    from quantized_block_sparse_b200 import sagesla as S
+    from quantized_block_sparse_b200.heads_parallel import HeadParallelSageSLA, local_heads
+
+    rank, world, local = rank_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_ranks(world, "nccl", dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    S.lib()
+    q, k, v = make_workload_qkv(wl)  # the same layer on every rank; each keeps its heads
+    ql, kl, vl = (local_heads(t, rank, world).contiguous() for t in (q, k, v))
+    qd, kd, vd = ql.to(dev), kl.to(dev), vl.to(dev)
+    layer = HeadParallelSageSLA(wl.B, wl.H, wl.N, wl.rho, wl.nu, rank, world, device=dev)
+    gather = not args.no_gather
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        layer(qd, kd, vd, gather=gather)
+    torch.cuda.synchronize(dev)
+    layer.check()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        out = layer(qd, kd, vd, gather=gather)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    step_ms = max_over_ranks_of(e0.elapsed_time(e1) / args.steps, world, dev)
+    layer.check()
+    # end to end: the rank's inputs from pinned host memory, the gathered output back
+    qh, kh, vh = (t.pin_memory() for t in (ql, kl, vl))
+    oh = torch.empty(tuple(out.shape), dtype=out.dtype).pin_memory()
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        for dst, src in zip((qd, kd, vd), (qh, kh, vh)):
+            dst.copy_(src, non_blocking=True)
+        o = layer(qd, kd, vd, gather=gather)
+        oh.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks_of(e0.elapsed_time(e1) / args.steps, world, dev)
+    ops = dense_equiv_ops(wl)
+    line = {
+        "metric": METRIC, "value": ops / (step_ms * 1e-3) / 1e12, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "int8 QK^T + bf16 PV (fp32 accumulate)", "data": "synthetic",
+        "config": dict(workload_config(wl), parallelism=(
+            f"heads split over {world} ranks (rank r: heads {layer.lo}..{layer.hi - 1} on rank "
+            f"{rank}); " + ("NCCL all-gather of the outputs each step" if gather else "no gather"))),
+        "e2e": {"value": ops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (qh, kh, vh)),
+                "d2h_bytes_per_step": oh.numel() * oh.element_size()},
+        "gpu_launches": None, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del layer
     if world > 1:
         dist.destroy_process_group()
     return 0
@@ -471,14 +601,25 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="480p", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="480p", choices=sorted(WORKLOADS) + ["sweep"],
+                    help="'sweep' runs the five sparsity-sweep points, one JSON line each")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--parallel", default="batch", choices=["batch", "heads"],
+                    help="batch: rank r runs batch element r (default, weak scaling); heads: one "
+                         "layer's heads split over the ranks (strong scaling)")
+    ap.add_argument("--no-gather", action="store_true",
+                    help="with --parallel heads: skip the all-gather of the outputs")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
-    wl = WORKLOADS[args.workload]
-    if args.impl == "reference":
-        return run_reference(args, wl)
-    return run_ours(args, wl)
+    names = [f"sweep_rho{r:g}" for r in SWEEP_RHOS] if args.workload == "sweep" else [args.workload]
+    rc = 0
+    for name in names:
+        wl = WORKLOADS[name]
+        if args.impl == "reference":
+            rc |= run_reference(args, wl)
+        else:
+            rc |= (run_heads if args.parallel == "heads" else run_ours)(args, wl)
+    return rc
 
 
 if __name__ == "__main__":
