@@ -11,7 +11,10 @@
 //     tensor-core instruction is a full M = 128 tcgen05.mma. pair_kernel chooses the
 //     pairs: blocks sharing many critical key blocks go together. The CTA walks the union
 //     of the two blocks' ascending critical lists; for a key block in only one list the
-//     P.V MMA masks the other half's rows (disable-output-lane mask).
+//     P.V MMA masks the other block's rows (disable-output-lane mask).
+//   * The two blocks' rows are interleaved in 16-row groups (block i0 in TMEM lanes
+//     32g..32g+15, block i1 in 32g+16..32g+31), so each block's softmax is spread over
+//     all four SM sub-partitions, also on steps where only one block is critical.
 //   * Warp-specialised:
 //     - warp 0, TMA producer: the pair's Q8 once; per union step one INT8 K tile (8 KB)
 //       into a 5-slot ring (with the step's block index, membership and k-scale beside
@@ -19,7 +22,11 @@
 //     - warp 1, one thread issues every tcgen05.mma: kind::i8 S = Q8 K8^T (M128 N64 K128,
 //       s32) into one of two 64-column TMEM score buffers, then kind::f16 O += P V with P
 //       read from TMEM (M128 N128 K64, fp32 O in TMEM). QK(t+1) is issued before waiting
-//       for P(t); P.V(t) as soon as the member halves have written P(t).
+//       for P(t); P.V(t) as soon as the member halves have written P(t). Each tcgen05
+//       instruction costs the issuing thread tens of cycles, so a step commits only twice:
+//       once after QK (s_full) and once after P.V (the V slot's v_empty, which also tells
+//       the rare rescale path that P.V has completed); the producer reuses a K slot once
+//       its QK's s_full phase and the softmax warps' metadata reads (k_empty) are done.
 //     - warps 2-9, softmax: two threads per query row (16-lane TMEM shapes, 16 keys each
 //       of two rows), scores dequantised by s_q * s_k * log2(e) through an exact
 //       magic-number int->float and packed f32x2 FMAs, exp2 on the SFU, P rounded to bf16
@@ -50,7 +57,7 @@ constexpr int kOffQ = 0;
 constexpr int kOffK = 16384;
 constexpr int kOffV = kOffK + kKStages * kKBytes;
 constexpr int kOffBar = kOffV + kVStages * kVBytes;
-constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 8 + 4 + 2 + 1 + 1;
+constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 8 + 4 + 1 + 1;
 constexpr int kOffMeta = kOffBar + 512;               // per-K-slot tile metadata (StageMeta)
 constexpr int kOffRowSum = kOffMeta + kKStages * 16;  // final row sums, [128]
 constexpr int kAttnSmem = kOffRowSum + 128 * 4 + 1024;  // ~106 KB: two CTAs per SM
@@ -306,8 +313,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   // step t-8, is then always complete, so a parity wait can never alias.
   uint64_t* s_full = v_empty + kVStages;
   uint64_t* p_full = s_full + 8;  // [half][buffer]
-  uint64_t* pv_done = p_full + 4;
-  uint64_t* o_full = pv_done + 2;
+  uint64_t* o_full = p_full + 4;
   uint64_t* lsum_bar = o_full + 1;  // final row sums written (all softmax threads)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lsum_bar + 1);
   StageMeta* meta = reinterpret_cast<StageMeta*>(smem + kOffMeta);
@@ -324,7 +330,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   }
   if (seg >= p.n_seg) return;  // past the head's last tile (whole CTA, before any barrier)
   const int2 pq = p.pairs[static_cast<size_t>(bh) * nB + seg * kPairSegment + tile];
-  const int i0 = pq.x, i1 = pq.y;  // rows 0-63: block i0; rows 64-127: block i1 (-1: none)
+  const int i0 = pq.x, i1 = pq.y;  // the pair (i1 = -1: block i0 alone)
 
   UnionWalk walk;
   walk.c0 = p.crit + (static_cast<size_t>(bh) * nB + i0) * p.k_c;
@@ -339,7 +345,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     mbar_init(smem_u32(q_full), 1);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(smem_u32(k_full + s), 1);
-      mbar_init(smem_u32(k_empty + s), 1 + kSoftmaxWarps);  // QK commit + one per softmax warp
+      mbar_init(smem_u32(k_empty + s), kSoftmaxWarps);  // every softmax warp has read the metadata
     }
     for (int s = 0; s < kVStages; ++s) {
       mbar_init(smem_u32(v_full + s), 1);
@@ -349,7 +355,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(p_full + b), 128);      // half 0 rows, buffer b
       mbar_init(smem_u32(p_full + 2 + b), 128);  // half 1 rows, buffer b
-      mbar_init(smem_u32(pv_done + b), 1);
     }
     mbar_init(smem_u32(o_full), 1);
     mbar_init(smem_u32(lsum_bar), 32 * kSoftmaxWarps);
@@ -372,9 +377,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     // One thread feeds both rings without blocking on either: K tiles (with the step's
     // metadata) run up to kKStages steps ahead of the V tiles.
     if (lane == 0) {
+      // rows interleaved in 16-row groups: tile rows 32g..32g+15 = block i0 rows 16g..16g+15,
+      // tile rows 32g+16..32g+31 = block i1 rows 16g..16g+15 (TMEM lane = tile row)
       mbar_expect_tx(smem_u32(q_full), 16384);
-      tma_load_3d(sQ, &tmQ, smem_u32(q_full), 0, i0 * 64, bh);
-      tma_load_3d(sQ + 8192, &tmQ, smem_u32(q_full), 0, (i1 >= 0 ? i1 : i0) * 64, bh);
+      const int i1r = i1 >= 0 ? i1 : i0;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        tma_load_3d(sQ + 4096 * g, &tmQ, smem_u32(q_full), 0, i0 * 64 + 16 * g, bh);
+        tma_load_3d(sQ + 4096 * g + 2048, &tmQ, smem_u32(q_full), 0, i1r * 64 + 16 * g, bh);
+      }
       int j, fl;
       bool have = walk.next(j, fl);  // k_c >= 1: at least one step
       int tK = 0, tV = 0, nsteps = -1;  // nsteps: known once the walk is exhausted
@@ -384,8 +395,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       for (;;) {
         bool progress = false;
         // K: as far ahead as the ring allows (and never more than kKStages beyond V)
+        // a K slot is free once every softmax warp has read its metadata (k_empty) and the
+        // QK^T of its previous step has completed (that step's s_full phase)
         while (have && tK < tV + kKStages &&
-               (tK < kKStages || mbar_test_wait(smem_u32(k_empty + ks), kph ^ 1))) {
+               (tK < kKStages ||
+                (mbar_test_wait(smem_u32(k_empty + ks), kph ^ 1) &&
+                 mbar_test_wait(smem_u32(s_full + ((tK - kKStages) & 7)), ((tK - kKStages) >> 3) & 1)))) {
           int jn, fln;
           const bool have_next = walk.next(jn, fln);
           meta[ks].j = j;
@@ -476,15 +491,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           }
         }
         tc_fence_after();
-        const uint32_t m01 = (fl & 1) ? 0u : 0xffffffffu;  // disable lanes 0-63 if half 0 is out
-        const uint32_t m23 = (fl & 2) ? 0u : 0xffffffffu;
+        // block i0 owns lanes 0-15 of every 32-lane group, block i1 lanes 16-31: a set bit
+        // disables that output lane
+        const uint32_t mk = ((fl & 1) ? 0u : 0x0000ffffu) | ((fl & 2) ? 0u : 0xffff0000u);
         const uint64_t dv = dv0 + kVDesc * vs;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16_ts_masked(taddr + kColO, taddr + 64 * b + 8 * kk, dv + 128 * kk, idesc_pv, 1u,
-                             m01, m01, m23, m23);
-        mma_commit(smem_u32(v_empty + vs));
-        mma_commit(smem_u32(pv_done + b));
+                             mk, mk, mk, mk);
+        mma_commit(smem_u32(v_empty + vs));  // V slot free, and P.V(u) complete (rescale)
         if (++vs == kVStages) {
           vs = 0;
           vph ^= 1;
@@ -506,7 +521,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_i8(taddr + 64 * b, dq + 2 * kk, dk + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
-        mma_commit(smem_u32(k_empty + s));
         mma_commit(smem_u32(s_full + (t & 7)));
         if (t >= 1 && !issue_pv(t - 1, prev_flags)) {
           ok = false;
@@ -525,17 +539,17 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     }
   } else {
     // ------------------------------------------------------------ softmax (warps 2-9)
-    // Warp w owns the 16 TMEM lanes LB = 32*(w%4) + 16*((w-2)/4) .. LB+15 (query rows of the
-    // 128-row tile); in the 16-lane load shape thread t holds rows LB + t/4 and LB + t/4 + 8,
-    // 16 keys each, and the four threads of a quad (t/4) share rows. Rows 0-63 are block i0,
-    // 64-127 block i1, so membership is warp-uniform. A warp whose half is not critical
-    // for a step skips it (the P.V MMA masks its rows).
+    // Warp w owns the 16 TMEM lanes LB = 32*(w%4) + 16*((w-2)/4) .. LB+15: rows 16*(w%4)..+15
+    // of block i0 for warps 2-5 and of block i1 for warps 6-9 (interleaved layout), so
+    // membership is warp-uniform. In the 16-lane load shape thread t holds rows LB + t/4
+    // and LB + t/4 + 8, 16 keys each; the four threads of a quad (t/4) share rows. A warp
+    // whose block is not critical for a step skips it (the P.V MMA masks its rows).
     const int wq = warp & 3;
     const int sub = (warp - 2) >> 2;
     const uint32_t lb = 32 * wq + 16 * sub;
     const int q = lane & 3;
     const int rr0 = static_cast<int>(lb) + (lane >> 2);  // rows rr0 and rr0 + 8
-    const int half = rr0 >> 6;
+    const int half = sub;  // lanes 32*wq + 16*sub .. +15 hold rows of block i0 (sub 0) or i1
     const int i = half ? i1 : i0;
     const float sq = (i >= 0) ? p.q_scale[static_cast<size_t>(bh) * nB + i] : 0.f;
     const uint32_t lane_off = lb << 16;
@@ -635,9 +649,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         tmem_st_16x128b_x8(taddr + lane_off + 64 * b, pk);  // P first: its registers die here
         if (rescale) {  // warp-uniform
           // O holds P.V of earlier steps: wait for the last issued P.V, then rescale rows.
-          if (t >= 1)
-            ok = mbar_wait(smem_u32(pv_done + ((t - 1) & 1)), ((t - 1) >> 1) & 1, &abort_flag,
-                           p.status);
+          if (t >= 1)  // P.V(t-1) complete: the v_empty phase of its V slot
+            ok = mbar_wait(smem_u32(v_empty + ((t - 1) % kVStages)), ((t - 1) / kVStages) & 1,
+                           &abort_flag, p.status);
           if (!__all_sync(0xffffffffu, ok)) {
             ok = false;
             break;
@@ -685,8 +699,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     // Epilogue layout: warp w reads its quadrant's 32 lanes (32x32b), one row per thread,
     // output columns [64*sub, 64*sub + 64).
     const int r = 32 * wq + lane;
-    const int ie = (r >> 6) ? i1 : i0;
-    const int tok = ie * 64 + (r & 63);
+    const int ie = (lane >> 4) ? i1 : i0;
+    const int tok = ie * 64 + 16 * wq + (lane & 15);
     const bool row_valid = (ie >= 0) && (tok < p.N);
     const uint32_t eoff = static_cast<uint32_t>(32 * wq) << 16;
     if (ok) {
@@ -805,7 +819,7 @@ cudaError_t launch_attention(const Dims& g, const int8_t* q8, const int8_t* k8,
                              cudaStream_t st) {
   const WsLayout L = ws_layout(g);
   CUtensorMap tmQ, tmK, tmV;
-  if (!make_tmap_3d(&tmQ, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kHeadDim, g.Npad, g.BH, 128, 64) ||
+  if (!make_tmap_3d(&tmQ, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kHeadDim, g.Npad, g.BH, 128, 16) ||
       !make_tmap_3d(&tmK, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kHeadDim, g.Npad, g.BH, 128, 64) ||
       !make_tmap_3d(&tmV, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim, g.N, g.BH, 64, 64))
     return cudaErrorInvalidValue;
