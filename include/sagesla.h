@@ -156,6 +156,32 @@ int sagesla_forward(const sagesla_shape* shape, const void* q, float sm_scale,
 int sagesla_check_status(const void* workspace, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * Backward pass ("TurboDiffusion Demystified", section "Pillar Two: Sparse-Linear
+ * Attention - SLA": the sparse-linear attention is trainable; section "Advanced Guide: How
+ * is TurboDiffusion Trained?"). The gradient of steps (1)-(7) for an upstream gradient dO,
+ * with the block lists held fixed (they are discrete) and the INT8 quantization read as
+ * the identity (straight through): scores Q~.K~^T in full precision, P not rounded. The
+ * smoothing mean depends on all of K, so dK sums to zero over tokens.
+ * ---------------------------------------------------------------------------------- */
+
+/* Bytes of device workspace sagesla_backward needs (it holds the status word, H, Z, the
+ * per-row softmax statistics, dH, dZ, their masked sums and small scratch). */
+size_t sagesla_backward_workspace_bytes(const sagesla_shape* shape);
+
+/* dQ, dK, dV (fp32 [B,H,N,d], rows t >= N untouched) for dout bf16 [B,H,N,d].
+ * Inputs: q, k, v bf16 [B,H,N,d] and sm_scale as given to the forward; k_mean, h, z from
+ * sagesla_prepare; crit_idx, marg_mask (and k_c, m) from sagesla_select (h, z, marg_mask
+ * may be NULL when m == 0). Arithmetic: bf16 operands (Q~, K~, V, dO, P, dS, phi, dn) with
+ * fp32 accumulation on tensor cores; softmax statistics, D = rowsum(dO o O_s) and the
+ * linear-branch denominators in fp32. Deterministic (fixed summation orders, no float
+ * atomics). The workspace status word records a timed-out device wait (check_status). */
+int sagesla_backward(const sagesla_shape* shape, const void* q, const void* k, const void* v,
+                     const void* dout, float sm_scale, const float* k_mean, const void* h,
+                     const float* z, const int32_t* crit_idx, int k_c, const void* marg_mask, int m,
+                     float* dq, float* dk, float* dv, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
+/* ------------------------------------------------------------------------------------
  * W8A8 block-wise INT8 linear layer ("TurboDiffusion Demystified", section "Pillar Three:
  * W8A8 Linear Layer Quantization": weights and activations of the linear layers in INT8,
  * block-wise at 128x128 granularity). Y = X W^T + bias with X [M, K] and W [N, K] each

@@ -257,6 +257,36 @@ int sagesla_forward(const sagesla_shape* shape, const void* q, float sm_scale, c
   return from_cuda(sgs::launch_attention(g, q8, k8, q_scale, k_scale, v, crit_idx, k_c, m, out, ws, st));
 }
 
+size_t sagesla_backward_workspace_bytes(const sagesla_shape* shape) {
+  Dims g;
+  if (make_dims(shape, &g) != SAGESLA_OK) return 0;
+  return sgs::backward_workspace_bytes(g);
+}
+
+int sagesla_backward(const sagesla_shape* shape, const void* q, const void* k, const void* v,
+                     const void* dout, float sm_scale, const float* k_mean, const void* h,
+                     const float* z, const int32_t* crit_idx, int k_c, const void* marg_mask, int m,
+                     float* dq, float* dk, float* dv, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  Dims g;
+  int rc = make_dims(shape, &g);
+  if (rc != SAGESLA_OK) return rc;
+  if (k_c < 1 || k_c > g.nB || m < 0 || m > g.nB - k_c) return SAGESLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, dout, k_mean, crit_idx, dq, dk, dv, workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return SAGESLA_ERR_INVALID_ARG;
+  if (m > 0) {
+    const void* lp[] = {h, z, marg_mask};
+    for (const void* p : lp)
+      if (!aligned16(p)) return SAGESLA_ERR_INVALID_ARG;
+  }
+  if (!(sm_scale > 0.f) || !isfinite(sm_scale)) return SAGESLA_ERR_INVALID_ARG;
+  if (workspace_bytes < sgs::backward_workspace_bytes(g)) return SAGESLA_ERR_INVALID_ARG;
+  return from_cuda(sgs::launch_backward(g, q, k, v, dout, sm_scale, k_mean, h, z, crit_idx, k_c,
+                                        marg_mask, m, dq, dk, dv, static_cast<char*>(workspace),
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 int sagesla_check_status(const void* workspace, void* stream) {
   if (!aligned16(workspace)) return SAGESLA_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SAGESLA_ERR_CUDA;

@@ -371,6 +371,40 @@ __global__ void __launch_bounds__(kLinThreads) linout_kernel(const __grid_consta
 
 }  // namespace
 
+// Sums of per-key-block states over a 0/1 block mask, per head: Hout[i] = sum_j M[i][j] h[j]
+// (bf16 [nB, d*d]) and Zout[i] = sum_j M[i][j] z[j] (fp32 [nB, d]); M bf16 [nB, nBp].
+// zb is scratch for the hi/lo split of z (bf16 [BH, nB, 2d]).
+cudaError_t launch_mask_gemm(const Dims& g, const void* mask, const void* h, const float* z,
+                             __nv_bfloat16* Hout, float* Zout, __nv_bfloat16* zb, int* status,
+                             cudaStream_t st) {
+  CUtensorMap tmA, tmB, tmZ;
+  if (!make_tmap_3d(&tmA, mask, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.nBp, g.nB, g.BH, 64, 128) ||
+      !make_tmap_3d(&tmB, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim * kHeadDim, g.nB, g.BH, 64,
+                    64) ||
+      !make_tmap_3d(&tmZ, zb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 2 * kHeadDim, g.nB, g.BH, 64, 64))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(hgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  if (e != cudaSuccess) return e;
+  {
+    TraceScope ts_("zb_kernel", st);
+    const size_t n4 = static_cast<size_t>(g.BH) * g.nB * kHeadDim / 4;
+    const int blocks = static_cast<int>((n4 + 255) / 256 < 4096 ? (n4 + 255) / 256 : 4096);
+    zb_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(z), reinterpret_cast<uint2*>(zb), n4);
+  }
+  {
+    TraceScope ts_("hgemm_kernel", st);
+    const int n_mt = (g.nB + 127) / 128;
+    const int n_tiles = (kHeadDim * kHeadDim / 256 + 1) * n_mt * g.BH;
+    int dev = 0, n_sm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = n_tiles < n_sm ? n_tiles : n_sm;
+    hgemm_kernel<<<grid, kGemmThreads, kGemmSmem, st>>>(tmA, tmB, tmZ, Hout, Zout, g.nB, n_mt, n_tiles,
+                                                         status);
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_linear(const Dims& g, const void* q, float sm_scale, const void* mask,
                           const int32_t* marg, int m, const void* h, const float* z, char* ws,
                           cudaStream_t st) {
@@ -382,39 +416,16 @@ cudaError_t launch_linear(const Dims& g, const void* q, float sm_scale, const vo
   __nv_bfloat16* Ol = reinterpret_cast<__nv_bfloat16*>(ws + L.Ol);
   __nv_bfloat16* Zb = reinterpret_cast<__nv_bfloat16*>(ws + L.Zb);
 
-  CUtensorMap tmA, tmB, tmZ, tmH, tmQ, tmO;
-  if (!make_tmap_3d(&tmA, mask, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.nBp, g.nB, g.BH, 64, 128) ||
-      !make_tmap_3d(&tmB, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim * kHeadDim, g.nB, g.BH, 64,
-                    64) ||
-      !make_tmap_3d(&tmZ, Zb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 2 * kHeadDim, g.nB, g.BH, 64, 64) ||
-      !make_tmap_3d(&tmH, Hbuf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim,
+  cudaError_t e = launch_mask_gemm(g, mask, h, z, Hbuf, Zbuf, Zb, status, st);
+  if (e != cudaSuccess) return e;
+  CUtensorMap tmH, tmQ, tmO;
+  if (!make_tmap_3d(&tmH, Hbuf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim,
                     static_cast<uint64_t>(g.nB) * kHeadDim, g.BH, 64, 128) ||
       !make_tmap_3d(&tmQ, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim, g.N, g.BH, 64, 64) ||
       !make_tmap_3d(&tmO, Ol, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim, g.N, g.BH, 64, 64))
     return cudaErrorInvalidValue;
-
-  cudaError_t e = cudaFuncSetAttribute(hgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
-  if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(linout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem);
   if (e != cudaSuccess) return e;
-
-  {
-    TraceScope ts_("zb_kernel", st);
-    const size_t n4 = static_cast<size_t>(g.BH) * g.nB * kHeadDim / 4;
-    const int blocks = static_cast<int>((n4 + 255) / 256 < 4096 ? (n4 + 255) / 256 : 4096);
-    zb_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(z), reinterpret_cast<uint2*>(Zb), n4);
-  }
-  {
-    TraceScope ts_("hgemm_kernel", st);
-    const int n_mt = (g.nB + 127) / 128;
-    const int n_tiles = (kHeadDim * kHeadDim / 256 + 1) * n_mt * g.BH;
-    int dev = 0, n_sm = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-    const int grid = n_tiles < n_sm ? n_tiles : n_sm;
-    hgemm_kernel<<<grid, kGemmThreads, kGemmSmem, st>>>(tmA, tmB, tmZ, Hbuf, Zbuf, g.nB, n_mt, n_tiles,
-                                                         status);
-  }
   {
     TraceScope ts_("linout_kernel", st);
     linout_kernel<<<dim3((g.nB + 1) / 2, g.BH), kLinThreads, kLinSmem, st>>>(tmH, tmQ, tmO, Zbuf, sm_scale,

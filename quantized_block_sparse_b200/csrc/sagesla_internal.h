@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -47,11 +48,21 @@ cudaError_t launch_select(const Dims& g, const float* q_bar, const float* k_bar,
 cudaError_t launch_linear(const Dims& g, const void* q, float sm_scale, const void* mask,
                           const int32_t* marg, int m, const void* h, const float* z, char* ws,
                           cudaStream_t st);
+cudaError_t launch_mask_gemm(const Dims& g, const void* mask, const void* h, const float* z,
+                             __nv_bfloat16* Hout, float* Zout, __nv_bfloat16* zb, int* status,
+                             cudaStream_t st);
 // attention.cu
 cudaError_t launch_attention(const Dims& g, const int8_t* q8, const int8_t* k8,
                              const float* q_scale, const float* k_scale, const void* v,
                              const int32_t* crit, int k_c, int m, void* out, char* ws,
                              cudaStream_t st);
+
+// backward.cu
+size_t backward_workspace_bytes(const Dims& g);
+cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const void* v,
+                            const void* dout, float sm_scale, const float* k_mean, const void* h,
+                            const float* z, const int32_t* crit, int k_c, const void* mask, int m,
+                            float* dq, float* dk, float* dv, char* ws, cudaStream_t st);
 
 // Opt-in launch tracing (api.cu): while enabled, a CUDA event pair is recorded on the
 // launch stream around every kernel launch, so per-kernel device time can be read back.

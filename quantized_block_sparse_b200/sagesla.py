@@ -60,6 +60,12 @@ def lib():
     L.sagesla_static_scratch_status.restype = ctypes.c_int
     L.sagesla_selftest_wait_timeout.argtypes = [_vp, ctypes.c_size_t, ctypes.c_uint, _vp]
     L.sagesla_selftest_wait_timeout.restype = ctypes.c_int
+    L.sagesla_backward_workspace_bytes.argtypes = [sp]
+    L.sagesla_backward_workspace_bytes.restype = ctypes.c_size_t
+    L.sagesla_backward.argtypes = ([sp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp,
+                                    ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, _vp, _vp,
+                                    ctypes.c_size_t, _vp])
+    L.sagesla_backward.restype = ctypes.c_int
     L.sagesla_w8a8_quantize.argtypes = [_vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp]
     L.sagesla_w8a8_quantize.restype = ctypes.c_int
     L.sagesla_w8a8_linear.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int,
@@ -297,3 +303,29 @@ def sagesla_w8a8_linear(x8, sx, w8, sw, bias=None, workspace=None, out=None, str
                                      M, N, K, _ptr(workspace), workspace.numel(), _stream(stream)),
            "sagesla_w8a8_linear")
     return y
+
+
+# ---------------------------------------------------------------- backward
+def sagesla_backward(q, k, v, dout, prep: Prepared, sel: Selection, sm_scale=None, workspace=None,
+                     stream=None):
+    """(dQ, dK, dV) fp32 [B,H,N,128] of the SageSLA output for upstream gradient dout (bf16),
+    with the block lists of `sel` held fixed and the quantization read straight through."""
+    B, H, N, d, nB = _dims(q)
+    for t in (q, k, v, dout):
+        assert t.dtype == torch.bfloat16 and t.is_cuda and t.is_contiguous() and t.shape == q.shape
+    sh = _shape(B, H, N, d)
+    if workspace is None:
+        n = lib().sagesla_backward_workspace_bytes(ctypes.byref(sh))
+        if n == 0:
+            raise SageSLAError("invalid shape")
+        workspace = torch.zeros(n, dtype=torch.uint8, device=q.device)
+    dq, dk, dv = (torch.empty(B, H, N, d, dtype=torch.float32, device=q.device) for _ in range(3))
+    c_s = softmax_scale(d) if sm_scale is None else float(sm_scale)
+    m = sel.m
+    _check(lib().sagesla_backward(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(dout), c_s,
+                                  _ptr(prep.k_mean), _ptr(prep.h) if m > 0 else None,
+                                  _ptr(prep.z) if m > 0 else None, _ptr(sel.crit), sel.k_c,
+                                  _ptr(sel.mask) if m > 0 else None, m, _ptr(dq), _ptr(dk), _ptr(dv),
+                                  _ptr(workspace), workspace.numel(), _stream(stream)),
+           "sagesla_backward")
+    return dq, dk, dv, workspace
