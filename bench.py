@@ -595,6 +595,134 @@ def run_heads(args, wl):
     return 0
 
 
+def _timed(fn, steps, warmup, stream):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def _kernel_times(fn, S):
+    """Per-kernel average device time (ms) of one call of fn, from the library's launch trace."""
+    import ctypes
+
+    import torch
+    L = S.lib()
+    L.sagesla_trace_enable(1)
+    fn()
+    torch.cuda.synchronize()
+    L.sagesla_trace_enable(0)
+    buf = ctypes.create_string_buffer(1 << 16)
+    L.sagesla_trace_read(buf, len(buf))
+    out, launches = {}, 0
+    for line in buf.value.decode().strip().splitlines():
+        name, cnt, tot = line.split()
+        out[name] = round(float(tot) / int(cnt), 5)
+        launches += int(cnt)
+    return out, launches
+
+
+def run_backward(args, wl):
+    """`--op backward`: sagesla_backward (dQ, dK, dV for an upstream gradient) on the workload."""
+    import torch
+
+    from quantized_block_sparse_b200 import sagesla as S
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    S.lib()
+    q, k, v = make_workload_qkv(wl)
+    do = torch.randn(*q.shape, generator=torch.Generator().manual_seed(9)).to(torch.bfloat16)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    eng = S.SageSLA(wl.B, wl.H, wl.N, wl.rho, wl.nu, device=dev)
+    eng(qd, kd, vd)
+    ws = S.sagesla_backward(qd, kd, vd, dod, eng.prep, eng.sel)[3]
+    fn = lambda: S.sagesla_backward(qd, kd, vd, dod, eng.prep, eng.sel, workspace=ws)  # noqa: E731
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    ms = _timed(fn, args.steps, args.warmup, torch.cuda.current_stream(dev))
+    clk = clocks.stop()
+    S.sagesla_check_status(ws)
+    kern, launches = _kernel_times(fn, S)
+    nB, k_c, n_neg, m = S.sagesla_counts(wl.B, wl.H, wl.N, wl.rho, wl.nu)
+    heads = wl.B * wl.H
+    gemm = 2.0 * 64 * 64 * 128
+    # algorithmic work: 5 GEMMs per critical pair (S, dP, dV, dK, dQ), the linear branch's
+    # phi(Q)H, dn H^T, phi(Q)^T dn per query block and phi(K)G, V G^T per key block, and the
+    # two masked sums H = M h and G = M^T dH over the marginal blocks
+    flops = heads * nB * k_c * 5 * gemm
+    if m > 0:
+        flops += heads * nB * (3 + 2) * 2.0 * 64 * 128 * 128 + 2 * heads * nB * m * 2.0 * 128 * 128
+    peaks, src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (ms * 1e-3) / 1e12
+    line = {"op": "backward", "metric": "SageSLA backward ms/call (dQ, dK, dV)", "value": ms,
+            "unit": "ms", "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
+            "dtype": "bf16 operands, fp32 accumulate (mma.sync tensor-core path)",
+            "data": "synthetic", "config": workload_config(wl), "kernels_ms": kern,
+            "gpu_launches": launches,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "note": f"algorithmic {flops / 1e12:.3f} TFLOP per call over the executed "
+                                 f"blocks; peak = {src} cuBLAS bf16 burst"},
+            "clocks": clk}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+W8A8_SHAPES = {  # Wan-1.3B linear layers at 480p: tokens x hidden 1536, FFN 8960
+    "qkv": (32760, 4608, 1536), "out": (32760, 1536, 1536), "ffn_up": (32760, 8960, 1536),
+    "ffn_down": (32760, 1536, 8960)}
+
+
+def run_w8a8(args):
+    """`--op w8a8`: the W8A8 block-wise INT8 linear layer on the Wan-1.3B 480p shapes."""
+    import torch
+
+    from quantized_block_sparse_b200 import sagesla as S
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    S.lib()
+    peaks, src = load_peaks()
+    peak_i8 = INT8_TO_BF16_RATE * float(peaks["bf16_tflops"])
+    g = torch.Generator(device=dev).manual_seed(0)
+    rc = 0
+    for name, (M, N, K) in W8A8_SHAPES.items():
+        x = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
+        w = (torch.randn(N, K, device=dev, generator=g) * 0.05).to(torch.bfloat16)
+        x8, sx = S.sagesla_w8a8_quantize(x)
+        w8, sw = S.sagesla_w8a8_quantize(w)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+        stream = torch.cuda.current_stream(dev)
+        t_gemm = _timed(lambda: S.sagesla_w8a8_linear(x8, sx, w8, sw, None, workspace=ws, out=y),  # noqa: E731
+                        args.steps, args.warmup, stream)
+        t_q = _timed(lambda: S.sagesla_w8a8_quantize(x), args.steps, args.warmup, stream)  # noqa: E731
+        S.sagesla_check_status(ws)
+        tops = 2.0 * M * N * K / (t_gemm * 1e-3) / 1e12
+        qgbs = (M * K * 3 + (M // 128 + 1) * (K // 128) * 4) / (t_q * 1e-3) / 1e9
+        line = {"op": "w8a8", "metric": "W8A8 block-wise INT8 linear (128x128 tiles) TOPS",
+                "value": tops, "unit": "TOPS", "higher_is_better": True, "steps": args.steps,
+                "warmup": args.warmup, "dtype": "int8 x int8 -> s32, fp32 scaling, bf16 out",
+                "data": "synthetic", "config": {"layer": name, "M": M, "N": N, "K": K},
+                "gemm_ms": t_gemm, "quantize_ms": t_q,
+                "roofline": {"bound": "tensor", "achieved": tops, "peak": peak_i8, "unit": "TOPS",
+                             "frac": tops / peak_i8, "traffic": None,
+                             "note": f"INT8 peak = {INT8_TO_BF16_RATE:g} x the {src} cuBLAS bf16 burst"},
+                "quantize_roofline": {"bound": "hbm", "achieved": qgbs,
+                                      "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                                      "frac": qgbs / float(peaks["hbm_gbs"])}}
+        print(json.dumps(line), flush=True)
+    return rc
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -609,9 +737,16 @@ def main():
                          "layer's heads split over the ranks (strong scaling)")
     ap.add_argument("--no-gather", action="store_true",
                     help="with --parallel heads: skip the all-gather of the outputs")
+    ap.add_argument("--op", default="attention", choices=["attention", "backward", "w8a8"],
+                    help="attention: the SageSLA forward path (default); backward: sagesla_backward; "
+                         "w8a8: the W8A8 linear layer on the Wan-1.3B shapes")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+    if args.op == "w8a8":
+        return run_w8a8(args)
     names = [f"sweep_rho{r:g}" for r in SWEEP_RHOS] if args.workload == "sweep" else [args.workload]
+    if args.op == "backward":
+        return max(run_backward(args, WORKLOADS[n]) for n in names)
     rc = 0
     for name in names:
         wl = WORKLOADS[name]

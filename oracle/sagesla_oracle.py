@@ -234,10 +234,29 @@ class Selection:
     neg: np.ndarray      # int32 [B,H,nB,n_neg] ascending
 
     def s_blk(self) -> np.ndarray:
-        """softmax_j of the fp32 logits, evaluated in fp64 (reported, not ranked on)."""
-        x = self.logits.astype(np.float64)
-        e = np.exp(x - x.max(axis=-1, keepdims=True))
-        return e / e.sum(axis=-1, keepdims=True)
+        """S_blk = softmax_j of the fp32 logits, in fp32 as the method states (max subtracted,
+        exp, row sum and divide each rounded to fp32). Reported, not ranked on: the lists
+        rank by the logit itself (the refinement of reading A7)."""
+        x = self.logits.astype(_F32)
+        e = np.exp((x - x.max(axis=-1, keepdims=True)).astype(_F32)).astype(_F32)
+        return (e / e.sum(axis=-1, keepdims=True, dtype=_F32)).astype(_F32)
+
+    def near_ties(self, rel: float = 1e-5) -> np.ndarray:
+        """bool [B,H,nB]: rows where fp32 S_blk cannot separate the two blocks on either side
+        of a class boundary (critical | marginal at position k_c, marginal | negligible at
+        nB - n_neg, in the logit order): equal values, or values within `rel` (relative).
+        There the method as stated in fp32 leaves the order open and the logit order (which
+        breaks such ties) is a refinement; these rows are the near-tie tally."""
+        p = self.s_blk().astype(np.float64)
+        nB = p.shape[-1]
+        order = np.argsort(self.rank, axis=-1)  # position -> block
+        ps = np.take_along_axis(p, order, axis=-1)
+        out = np.zeros(p.shape[:-1], dtype=bool)
+        for pos in (self.k_c, nB - self.n_neg):
+            if 0 < pos < nB:
+                a, b = ps[..., pos - 1], ps[..., pos]
+                out |= (a - b) <= rel * a
+        return out
 
     def marg_mask(self) -> np.ndarray:
         nB = self.logits.shape[-1]

@@ -113,14 +113,10 @@ def compare_lists(g, sel, heads=slice(None)):
     np.testing.assert_array_equal(gmask[..., :nB][ok_rows], sel.marg_mask()[ok_rows])
     assert not gmask[..., nB:].any()
     near = 0
+    ties = sel.near_ties(NEAR_TIE_REL)
     for idx in bad:
         idx = tuple(idx)
-        p = np.sort(sel.s_blk()[idx])[::-1]
-        ok = False
-        for kpos in (sel.k_c, nB - sel.n_neg):
-            if 0 < kpos < nB and (p[kpos - 1] - p[kpos]) / p[kpos - 1] < NEAR_TIE_REL:
-                ok = True
-        assert ok, f"list mismatch that is not a near-tie at row {idx}"
+        assert ties[idx], f"list mismatch that is not a near-tie at row {idx}"
         near += 1
     return near
 

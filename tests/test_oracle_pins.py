@@ -226,16 +226,21 @@ def test_select_ties_go_to_lower_index():
 
 
 def test_ranking_by_logit_equals_ranking_by_sblk():
-    q, k, v = make_qkv(1, 2, (4, 16, 16), seed=1)
-    prep = O.prepare(f32(q), f32(k))
-    sel = O.select(prep.q_bar, prep.k_bar, 0.25, 0.25)
-    p = sel.s_blk()
-    np.testing.assert_allclose(p.sum(-1), 1.0, rtol=1e-12)
-    for idx in np.ndindex(1, 2, 16):
-        order = np.argsort(-p[idx], kind="stable")
-        if not np.array_equal(np.sort(order[:sel.k_c]), sel.crit[idx]):
-            a, b_ = p[idx][order[sel.k_c - 1]], p[idx][order[sel.k_c]]
-            assert (a - b_) / a < 1e-5  # only a near-tie may differ
+    # Ranking by the fp32 S_blk (stable: ties to the lower index) gives the logit lists at
+    # both class boundaries except on near-tie rows, where fp32 S_blk leaves the order open.
+    for seed, grid in ((1, (4, 16, 16)), (2, (6, 20, 24))):
+        q, k, v = make_qkv(1, 2, grid, seed=seed)
+        prep = O.prepare(f32(q), f32(k))
+        sel = O.select(prep.q_bar, prep.k_bar, 0.25, 0.25)
+        p = sel.s_blk()
+        nB = p.shape[-1]
+        assert np.abs(p.astype(np.float64).sum(-1) - 1.0).max() <= nB * 2.0 ** -23
+        ties = sel.near_ties(1e-5)
+        for idx in np.ndindex(*p.shape[:-1]):
+            order = np.argsort(-p[idx], kind="stable")
+            same = (np.array_equal(np.sort(order[:sel.k_c]), sel.crit[idx]) and
+                    np.array_equal(np.sort(order[nB - sel.n_neg:]), sel.neg[idx]))
+            assert same or ties[idx], idx
 
 
 # ------------------------------------------------------------------ steps 5-7
@@ -428,3 +433,63 @@ def test_no_marginal_blocks_gives_zero_linear_term():
     assert sel.m == 0
     _, Os, Ol, _ = O.forward(prep, f32(v), sel, return_parts=True)
     assert (Ol == 0).all()
+
+
+# ---------------------------------------------------------------- S_blk in fp32, near ties
+def _sel_from_logits(logit_rows, rho, nu):
+    """A selection whose block logits are exactly the given values: q_bar = e_0 and
+    k_bar[j] = logit_j e_0, so each fused multiply-add chain returns logit_j unrounded."""
+    L = np.asarray(logit_rows, dtype=np.float32)
+    nQ, nK = L.shape
+    d = 4
+    qb = np.zeros((1, 1, nQ, d), dtype=np.float32)
+    qb[..., 0] = 1.0
+    kb = np.zeros((1, 1, nK, d), dtype=np.float32)
+    kb[0, 0, :, 0] = L[0]
+    sels = []
+    for r in range(nQ):
+        kb[0, 0, :, 0] = L[r]
+        sels.append(O.select(qb[:, :, r:r + 1], kb, rho, nu))
+    return sels
+
+
+def test_s_blk_is_an_fp32_softmax():
+    sel = _sel_from_logits([[3.0, 1.0, 0.5, -2.0, 0.0, 1.5, -1.0, 2.0]], 0.25, 0.25)[0]
+    p = sel.s_blk()
+    assert p.dtype == np.float32
+    x = sel.logits[0, 0, 0].astype(np.float64)
+    ref = np.exp(x - x.max()) / np.exp(x - x.max()).sum()
+    assert np.abs(p[0, 0, 0] - ref).max() <= 8 * 2.0 ** -24  # a few fp32 roundings
+    assert abs(float(p.astype(np.float64).sum()) - 1.0) <= 8 * 2.0 ** -24
+
+
+def test_near_ties_at_both_boundaries():
+    # nB = 8, rho = 0.25 -> k_c = 2, nu = 0.25 -> n_neg = 2: boundaries after positions 2 and 6
+    apart = [5.0, 4.0, 3.0, 2.0, 1.0, 0.0, -1.0, -2.0]
+    sep, = _sel_from_logits([apart], 0.25, 0.25)
+    assert not sep.near_ties().any()
+    # equal logits across the critical boundary: a tie the logit order breaks by index
+    tie_c, = _sel_from_logits([[5.0, 4.0, 4.0, 2.0, 1.0, 0.0, -1.0, -2.0]], 0.25, 0.25)
+    assert tie_c.near_ties().all()
+    assert tie_c.crit[0, 0, 0].tolist() == [0, 1]  # the lower index of the tied pair is critical
+    # logits 1e-7 apart at the negligible boundary: distinct logits, fp32 S_blk within 1e-5
+    close, = _sel_from_logits([[5.0, 4.0, 3.0, 2.0, 1.0, -1.0, -1.0000001, -2.0]], 0.25, 0.25)
+    assert close.logits[0, 0, 0, 5] > close.logits[0, 0, 0, 6]
+    assert close.near_ties().all()
+    # far below the row max fp32 S_blk underflows to 0 for both neighbours: still ranked by logit
+    under, = _sel_from_logits([[0.0, -1.0, -2.0, -3.0, -4.0, -300.0, -301.0, -302.0]], 0.25, 0.25)
+    assert under.s_blk()[0, 0, 0, 5] == 0.0 and under.s_blk()[0, 0, 0, 6] == 0.0
+    assert under.near_ties().all()
+    assert under.neg[0, 0, 0].tolist() == [6, 7]  # -301 and -302, the two smallest logits
+
+
+def test_near_tie_tally_on_the_480p_sample():
+    # The tally the method's fp32 S_blk leaves open on two heads of the 480p workload (seed 0):
+    # rows where the blocks on either side of a class boundary are within 1e-5 relative.
+    from quantized_block_sparse_b200.inputs import make_qkv
+    q, k, _ = make_qkv(1, 2, (21, 30, 52), seed=0)
+    prep = O.prepare(q.float().numpy(), k.float().numpy())
+    sel = O.select(prep.q_bar, prep.k_bar, 0.10, 0.45)
+    ties = sel.near_ties(1e-5)
+    assert ties.shape == (1, 2, 512)
+    assert int(ties.sum()) == 30  # of 1024 rows; none is an exact fp32 tie
