@@ -33,6 +33,7 @@ namespace w8 {
 
 constexpr int kTile = 128;
 constexpr int kStages = 4;
+constexpr int kParts = 4;  // TMEM partial buffers (128 columns each): the MMA runs up to 3 K tiles ahead
 constexpr int kStageBytes = 2 * kTile * kTile;  // A and B K tiles, int8, K-major SW128
 constexpr int kThreads = 320;
 constexpr int kMaxKT = 128;                     // K <= 16384
@@ -140,9 +141,9 @@ __global__ void __launch_bounds__(kThreads, 1) w8a8_gemm_kernel(const __grid_con
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
-  uint64_t* pfull = bars + 2 * kStages;  // [2] partial sum of a K tile ready (MMA commit)
-  uint64_t* pfree = pfull + 2;           // [2] partial read and re-armed (256 arrivals)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pfree + 2);
+  uint64_t* pfull = bars + 2 * kStages;  // [kParts] partial sum of a K tile ready (MMA commit)
+  uint64_t* pfree = pfull + kParts;      // [kParts] partial read and re-armed (256 arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pfree + kParts);
   float* sscale = reinterpret_cast<float*>(smem + kStages * kStageBytes + 256);  // [8][kMaxKT]
   __shared__ int abort_flag;
 
@@ -155,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1) w8a8_gemm_kernel(const __grid_con
       mbar_init(smem_u32(full + s), 1);
       mbar_init(smem_u32(empty + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kParts; ++b) {
       mbar_init(smem_u32(pfull + b), 1);
       mbar_init(smem_u32(pfree + b), 256);
     }
@@ -163,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1) w8a8_gemm_kernel(const __grid_con
     prefetch_tmap(&tmX);
     prefetch_tmap(&tmW);
   }
-  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 256);
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 128 * kParts);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -198,8 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1) w8a8_gemm_kernel(const __grid_con
       bool ok = true;
       for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
         for (int kb = 0; kb < nKT; ++kb, ++it) {
-          const int s = it % kStages, b = it & 1;
-          if (!mbar_wait(smem_u32(pfree + b), (it >> 1) & 1, &abort_flag, status) ||
+          const int s = it % kStages, b = it % kParts;
+          if (!mbar_wait(smem_u32(pfree + b), (it / kParts) & 1, &abort_flag, status) ||
               !mbar_wait(smem_u32(full + s), (it / kStages) & 1, &abort_flag, status)) {
             ok = false;
             break;
@@ -224,14 +225,14 @@ __global__ void __launch_bounds__(kThreads, 1) w8a8_gemm_kernel(const __grid_con
     const uint32_t lane_base = taddr + (static_cast<uint32_t>(32 * q) << 16) + 64 * h;
     float* my_scale = sscale + e * kMaxKT;
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kParts; ++b) {
       tmem_st32_fill(lane_base + 128 * b, kMagicBits);
       tmem_st32_fill(lane_base + 128 * b + 32, kMagicBits);
     }
     tmem_wait_st();
     tc_fence_before();
-    mbar_arrive(smem_u32(pfree + 0));
-    mbar_arrive(smem_u32(pfree + 1));
+#pragma unroll
+    for (int b = 0; b < kParts; ++b) mbar_arrive(smem_u32(pfree + b));
     const uint64_t neg_magic = f2pack(-12582912.f, -12582912.f);  // -(1.5 * 2^23)
     int it = 0;
     bool ok = true;
@@ -245,8 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1) w8a8_gemm_kernel(const __grid_con
 #pragma unroll
       for (int c = 0; c < 32; ++c) acc[c] = 0ull;
       for (int kb = 0; kb < nKT; ++kb, ++it) {
-        const int b = it & 1;
-        ok = mbar_wait(smem_u32(pfull + b), (it >> 1) & 1, &abort_flag, status);
+        const int b = it % kParts;
+        ok = mbar_wait(smem_u32(pfull + b), (it / kParts) & 1, &abort_flag, status);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
@@ -254,6 +255,9 @@ __global__ void __launch_bounds__(kThreads, 1) w8a8_gemm_kernel(const __grid_con
         tc_fence_after();
         const float s = my_scale[kb];
         const uint64_t s2 = f2pack(s, s);
+        // This thread's 64 columns in two halves; the buffer is re-armed and released after
+        // the second load, before that half's arithmetic, so the MMAs of the next K tiles
+        // (up to kParts - 1 ahead) overlap the scaling.
         uint32_t r[32];
         tmem_ld32_sync(lane_base + 128 * b, r);  // columns 0-31 of this thread's half
 #pragma unroll
@@ -262,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) w8a8_gemm_kernel(const __grid_con
           acc[c] = fma2(s2, xv, acc[c]);
         }
         tmem_ld32_sync(lane_base + 128 * b + 32, r);  // columns 32-63
-        tmem_st32_fill(lane_base + 128 * b, kMagicBits);  // re-arm the buffer for K tile it + 2
+        tmem_st32_fill(lane_base + 128 * b, kMagicBits);  // re-arm for K tile it + kParts
         tmem_st32_fill(lane_base + 128 * b + 32, kMagicBits);
         tmem_wait_st();
         tc_fence_before();
@@ -302,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) w8a8_gemm_kernel(const __grid_con
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(taddr, 256);
+  if (warp == 1) tmem_dealloc(taddr, 128 * kParts);
 }
 
 }  // namespace w8
