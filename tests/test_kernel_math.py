@@ -81,8 +81,10 @@ PREP = os.path.join(os.path.dirname(SRC), "prepare.cu")
 
 def _prep_threshold():
     text = open(PREP).read()
-    body = text[text.index("uint32_t quant_byte("):]
-    return F32(float(re.search(r"fabsf\(e\) > ([0-9.]+)f", body).group(1)))
+    body = text[text.index("uint64_t quant_pair("):]
+    m = re.search(r"fabsf\(e\.x\) > ([0-9.]+)f \|\| fabsf\(e\.y\) > ([0-9.]+)f", body)
+    assert m.group(1) == m.group(2)  # both lanes of the pair use one band
+    return F32(float(m.group(1)))
 
 
 def quant_byte_replay(x, s):
