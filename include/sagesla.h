@@ -141,8 +141,10 @@ int sagesla_select(const sagesla_shape* shape, const float* q_bar, const float* 
  *          computed as one GEMM with marg_mask; marg_idx (the same set as a list) is
  *          checked for alignment but not read (it may be NULL when m == 0).
  * Output : out bf16 [B,H,N,d] (rows t >= N are not touched).
+ * O_l = phi(Q~) H_i / (phi(Q~) . Z_i) is formed inside the attention kernel and added to
+ * O_s in fp32, so the output is rounded to bf16 once.
  * workspace: at least sagesla_workspace_bytes(shape) bytes; forward keeps H, Z, z in
- *          bf16, O_l and the query-block pairing of the attention tiles there. */
+ *          bf16 and the query-block pairing of the attention tiles there. */
 int sagesla_forward(const sagesla_shape* shape, const void* q, float sm_scale,
                     const int8_t* q8, const int8_t* k8, const float* q_scale,
                     const float* k_scale, const void* v, const int32_t* crit_idx, int k_c,

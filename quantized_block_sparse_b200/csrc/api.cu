@@ -32,8 +32,6 @@ WsLayout ws_layout(const Dims& g) {
   off = align256(off + static_cast<size_t>(g.BH) * g.nB * 8);
   L.pair_counts = off;
   off = align256(off + static_cast<size_t>(g.BH) * ((g.nB + 63) / 64) * 4);
-  L.Ol = off;
-  off = align256(off + static_cast<size_t>(g.BH) * g.N * kHeadDim * 2);
   L.total = off;
   return L;
 }
@@ -252,9 +250,10 @@ int sagesla_forward(const sagesla_shape* shape, const void* q, float sm_scale, c
   if (workspace_bytes < sgs::ws_layout(g).total) return SAGESLA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
-  cudaError_t e = sgs::launch_linear(g, q, sm_scale, marg_mask, marg_idx, m, h, z, ws, st);
+  cudaError_t e = sgs::launch_linear(g, marg_mask, m, h, z, ws, st);
   if (e != cudaSuccess) return SAGESLA_ERR_CUDA;
-  return from_cuda(sgs::launch_attention(g, q8, k8, q_scale, k_scale, v, crit_idx, k_c, m, out, ws, st));
+  return from_cuda(sgs::launch_attention(g, q, sm_scale, q8, k8, q_scale, k_scale, v, crit_idx, k_c, m,
+                                         out, ws, st));
 }
 
 size_t sagesla_backward_workspace_bytes(const sagesla_shape* shape) {

@@ -1,5 +1,5 @@
 // attention.cu - block-sparse INT8 attention over the critical key blocks, merged with the
-// linear-branch output.
+// linear-attention term of the marginal blocks.
 //
 // Method: "TurboDiffusion Demystified", section "Pillar One: Low-Bit Attention
 // Acceleration - SageAttention" (Q K^T on INT8 tensor cores) and section "Pillar Two:
@@ -33,7 +33,13 @@
 //       and written over the row's score columns.
 //   * The running max m is raised only when a tile's partial sum of 2^(s - m) leaves
 //     [0, 2^24]; only then is the exact tile max taken and O rescaled in TMEM.
-//   * Epilogue: O_s = O / l, plus the linear-branch O_l, rounded once to bf16.
+//   * Linear branch (marginal blocks, when there are any): after a CTA's last step the
+//     softmax warps write phi(Q~) of its 128 rows (recomputed from Q) as a K-major bf16
+//     A tile over the Q8 tile and K slots 0-1, with each row's phi(Q~) . Z_i; the producer
+//     streams H_i0 and H_i1 through the V ring as four 64 x 128 chunks; the MMA thread
+//     forms phi(Q~) H_i in TMEM columns [0, 128) (freed by the last P.V), each block's
+//     rows alone through the lane mask. O_l never goes to memory.
+//   * Epilogue: O = O / l + (phi(Q~) H_i) / (phi(Q~) . Z_i) in fp32, rounded once to bf16.
 // Every mbarrier wait is bounded (see sm100_primitives.cuh) and never traps.
 #include <climits>
 
@@ -60,7 +66,12 @@ constexpr int kOffBar = kOffV + kVStages * kVBytes;
 constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 8 + 4 + 1 + 1;
 constexpr int kOffMeta = kOffBar + 512;               // per-K-slot tile metadata (StageMeta)
 constexpr int kOffRowSum = kOffMeta + kKStages * 16;  // final row sums, [128]
-constexpr int kAttnSmem = kOffRowSum + 128 * 4 + 1024;  // ~106 KB: two CTAs per SM
+constexpr int kOffDen = kOffRowSum + 128 * 4;          // linear-branch denominator halves, [2][128]
+constexpr int kAttnSmem = kOffDen + 2 * 128 * 4 + 1024;  // ~107 KB: two CTAs per SM
+// After the last Q K^T, the Q8 tile and K slots 0-1 ([0, 32 KB)) hold the phi(Q~) A tile of
+// the linear branch: two 64-channel halves, 128 rows x 128 B each, K-major, 128-byte swizzle.
+constexpr int kOffPhi = 0;
+static_assert(kOffK + 2 * kKBytes == 32768 && kKStages >= 2, "phi(Q~) tile must fit over Q8 + 2 K slots");
 static_assert(kNumBars * 8 + 4 <= kOffMeta - kOffBar, "barriers + TMEM slot overflow");
 static_assert(2 * (kAttnSmem + 1024) <= 233472, "two CTAs per SM must fit in shared memory");
 constexpr int kSoftmaxWarps = 8;
@@ -98,7 +109,10 @@ struct AttnParams {
   const float* q_scale;
   const float* k_scale;
   const int32_t* crit;
-  const __nv_bfloat16* Ol;  // nullptr when there is no marginal block
+  const __nv_bfloat16* q;   // bf16 Q [BH][N][d] (linear branch; nullptr when m == 0)
+  const float* Z;           // Z_i fp32 [BH][nB][d]
+  const __nv_bfloat16* H;   // H_i bf16 [BH][nB][d][d] (L2 prefetch only)
+  float c_s;
   __nv_bfloat16* out;
   int* status;
   int N, nB, k_c, n_seg;
@@ -295,9 +309,21 @@ __device__ __forceinline__ void mma_bf16_ts_masked(uint32_t d_tmem, uint32_t a_t
       "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate), "r"(m0), "r"(m1), "r"(m2), "r"(m3));
 }
 
+// Both operands in shared memory, with the same disable-output-lane mask.
+__device__ __forceinline__ void mma_bf16_ss_masked(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                                   uint32_t idesc, uint32_t accumulate,
+                                                   uint32_t m0, uint32_t m1, uint32_t m2,
+                                                   uint32_t m3) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(m0), "r"(m1), "r"(m2), "r"(m3));
+}
+
 __global__ void __launch_bounds__(kAttnThreads, 2)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, AttnParams p) {
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmH,
+                AttnParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -318,6 +344,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lsum_bar + 1);
   StageMeta* meta = reinterpret_cast<StageMeta*>(smem + kOffMeta);
   float* rowsum = reinterpret_cast<float*>(smem + kOffRowSum);
+  float* denp = reinterpret_cast<float*>(smem + kOffDen);
   __shared__ int abort_flag;
 
   const int pr = blockIdx.x, bh = blockIdx.y;
@@ -331,6 +358,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   if (seg >= p.n_seg) return;  // past the head's last tile (whole CTA, before any barrier)
   const int2 pq = p.pairs[static_cast<size_t>(bh) * nB + seg * kPairSegment + tile];
   const int i0 = pq.x, i1 = pq.y;  // the pair (i1 = -1: block i0 alone)
+  // Linear branch: H_i0 (and H_i1) enter the V ring after the last V tile as 16 KB chunks
+  // of 64 channels x 128 columns: chunk u is rows [64*(u&1), +64) of H of block u>>1.
+  const bool lin = p.q != nullptr;
+  const int nH = lin ? (i1 >= 0 ? 4 : 2) : 0;
 
   UnionWalk walk;
   walk.c0 = p.crit + (static_cast<size_t>(bh) * nB + i0) * p.k_c;
@@ -362,6 +393,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
+    if (lin) prefetch_tmap(&tmH);
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
   tc_fence_before();
@@ -391,7 +423,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       int tK = 0, tV = 0, nsteps = -1;  // nsteps: known once the walk is exhausted
       int ks = 0, kph = 0, vs = 0, vph = 0;
       unsigned long long t_idle = 0;
-      bool aborted = false;
       for (;;) {
         bool progress = false;
         // K: as far ahead as the ring allows (and never more than kKStages beyond V)
@@ -413,18 +444,39 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             ks = 0;
             kph ^= 1;
           }
-          if (!have_next) nsteps = tK;
+          if (!have_next) {
+            nsteps = tK;
+            if (lin) {  // the linear branch's H tiles and Q rows, needed at the end of the walk
+              for (int b = 0; b < (i1 >= 0 ? 2 : 1); ++b) {
+                const int ib = b ? i1 : i0;
+                prefetch_l2(p.H + (static_cast<size_t>(bh) * nB + ib) * (kHeadDim * kHeadDim),
+                            kHeadDim * kHeadDim * 2);
+                const int rows = min(64, p.N - ib * 64);
+                prefetch_l2(p.q + (static_cast<size_t>(bh) * p.N + ib * 64) * kHeadDim,
+                            static_cast<uint32_t>(rows) * kHeadDim * 2);
+              }
+            }
+          }
           have = have_next;
           j = jn;
           fl = fln;
           progress = true;
         }
-        // V: the next step whose K has been issued, once its slot is free
-        if (tV < tK && (tV < kVStages || mbar_test_wait(smem_u32(v_empty + vs), vph ^ 1))) {
-          const int jv = meta[tV % kKStages].j;  // K slot of step tV: not reused before V(tV)
+        // V: the next step whose K has been issued, once its slot is free; after the last
+        // step, the linear branch's H chunks take the same ring
+        const bool v_next = tV < tK || (nsteps >= 0 && tV < nsteps + nH);
+        if (v_next && (tV < kVStages || mbar_test_wait(smem_u32(v_empty + vs), vph ^ 1))) {
           mbar_expect_tx(smem_u32(v_full + vs), kVBytes);
-          tma_load_3d(sV + vs * kVBytes, &tmV, smem_u32(v_full + vs), 0, jv * 64, bh);
-          tma_load_3d(sV + vs * kVBytes + 8192, &tmV, smem_u32(v_full + vs), 64, jv * 64, bh);
+          if (tV < tK) {
+            const int jv = meta[tV % kKStages].j;  // K slot of step tV: not reused before V(tV)
+            tma_load_3d(sV + vs * kVBytes, &tmV, smem_u32(v_full + vs), 0, jv * 64, bh);
+            tma_load_3d(sV + vs * kVBytes + 8192, &tmV, smem_u32(v_full + vs), 64, jv * 64, bh);
+          } else {
+            const int u = tV - nsteps;
+            const int crow = ((u >> 1) ? i1 : i0) * kHeadDim + 64 * (u & 1);
+            tma_load_3d(sV + vs * kVBytes, &tmH, smem_u32(v_full + vs), 0, crow, bh);
+            tma_load_3d(sV + vs * kVBytes + 8192, &tmH, smem_u32(v_full + vs), 64, crow, bh);
+          }
           ++tV;
           if (++vs == kVStages) {
             vs = 0;
@@ -432,16 +484,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           }
           progress = true;
         }
-        if (nsteps >= 0 && tV == nsteps) break;
+        if (nsteps >= 0 && tV == nsteps + nH) break;
         if (progress) {
           t_idle = 0;
           continue;
         }
         // nothing to issue: sleep on the V slot we need next (the usual blocker)
-        if (tV < tK && tV >= kVStages) mbar_try_wait_suspend(smem_u32(v_empty + vs), vph ^ 1, 2000u);
+        if (v_next && tV >= kVStages) mbar_try_wait_suspend(smem_u32(v_empty + vs), vph ^ 1, 2000u);
         else if (tK >= kKStages) mbar_try_wait_suspend(smem_u32(k_empty + ks), kph ^ 1, 2000u);
         if (abort_flag) {
-          aborted = true;
           break;
         }
         const unsigned long long now = globaltimer();
@@ -450,11 +501,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         } else if (now - t_idle > kWaitLimitNs) {
           abort_flag = 1;
           atomicOr(p.status, kStatusTimeout);
-          aborted = true;
           break;
         }
       }
-      if (aborted || abort_flag) {  // let the copies in flight land before exit
+      {  // every copy issued lands before the CTA exits (already true unless a wait gave up)
         mbar_drain(smem_u32(q_full), 0, p.status);
         for (int u = max(0, tK - kKStages); u < tK; ++u)
           mbar_drain(smem_u32(k_full + (u % kKStages)), (u / kKStages) & 1, p.status);
@@ -534,6 +584,32 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         }
       }
       if (ok && t >= 1) ok = issue_pv(t - 1, prev_flags);
+      if (ok && lin) {
+        // Linear branch into TMEM columns [0, 128) (free once the last P.V has read P, which
+        // issue order guarantees): phi(Q~) (written by the softmax warps, lsum_bar) times
+        // the H chunks from the V ring, each block's rows alone (the other's lanes masked).
+        ok = mbar_wait(smem_u32(lsum_bar), 0, &abort_flag, p.status);
+        const uint64_t da = make_sdesc(smem_u32(smem + kOffPhi), 16, 1024);
+        for (int u = 0; u < nH && ok; ++u) {
+          if (!mbar_wait(smem_u32(v_full + vs), vph, &abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t mk = (u >> 1) ? 0x0000ffffu : 0xffff0000u;
+          const uint64_t a = da + static_cast<uint64_t>((u & 1) * (16384 >> 4));
+          const uint64_t dv = dv0 + kVDesc * vs;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss_masked(taddr, a + 2 * kk, dv + 128 * kk, idesc_pv, ((u & 1) | kk) != 0 ? 1u : 0u,
+                               mk, mk, mk, mk);
+          mma_commit(smem_u32(v_empty + vs));
+          if (++vs == kVStages) {
+            vs = 0;
+            vph ^= 1;
+          }
+        }
+      }
       mma_commit(smem_u32(o_full));
       mbar_drain(smem_u32(o_full), 0, p.status);
     }
@@ -691,51 +767,73 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       rowsum[rr0] = l0;
       rowsum[rr0 + 8] = l1;
     }
-    mbar_arrive(smem_u32(lsum_bar));
-    ok = ok && mbar_wait(smem_u32(lsum_bar), 0, &abort_flag, p.status);
-    ok = ok && mbar_wait(smem_u32(o_full), 0, &abort_flag, p.status);
-    ok = __all_sync(0xffffffffu, ok);
-    tc_fence_after();
     // Epilogue layout: warp w reads its quadrant's 32 lanes (32x32b), one row per thread,
     // output columns [64*sub, 64*sub + 64).
     const int r = 32 * wq + lane;
     const int ie = (lane >> 4) ? i1 : i0;
     const int tok = ie * 64 + 16 * wq + (lane & 15);
     const bool row_valid = (ie >= 0) && (tok < p.N);
+    if (lin && ok) {
+      // phi(Q~) of this row's channels [64*sub, +64) into the A tile over Q8 and K slots 0-1,
+      // free once every Q K^T has completed (the last step's S is ready), and this half of
+      // the denominator phi(Q~).Z_i with the bf16-rounded phi the tensor core sees.
+      if (t >= 1) ok = mbar_wait(smem_u32(s_full + ((t - 1) & 7)), ((t - 1) >> 3) & 1, &abort_flag, p.status);
+      const uint32_t tile = smem_u32(smem + kOffPhi) + sub * 16384;
+      float dacc = 0.f;
+      if (row_valid) {
+        const uint4* qr = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(bh) * p.N + tok) * kHeadDim + 64 * sub);
+        const float4* zr = reinterpret_cast<const float4*>(p.Z + (static_cast<size_t>(bh) * nB + ie) * kHeadDim + 64 * sub);
+        uint4 qv[8];
+#pragma unroll
+        for (int cb = 0; cb < 8; ++cb) qv[cb] = __ldg(qr + cb);
+#pragma unroll
+        for (int cb = 0; cb < 8; ++cb) {
+          const float4 z0 = __ldg(zr + 2 * cb), z1 = __ldg(zr + 2 * cb + 1);
+          const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+          uint32_t w[4] = {qv[cb].x, qv[cb].y, qv[cb].z, qv[cb].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = __fmul_rn(__uint_as_float(w[e] << 16), p.c_s);
+            const float x1 = __fmul_rn(__uint_as_float(w[e] & 0xffff0000u), p.c_s);
+            w[e] = pack_bf16x2(x0 > 0.f ? x0 + 1.f : ex2_approx(x0 * kLog2e),
+                               x1 > 0.f ? x1 + 1.f : ex2_approx(x1 * kLog2e));
+            dacc = fmaf(__uint_as_float(w[e] << 16), zz[2 * e], dacc);
+            dacc = fmaf(__uint_as_float(w[e] & 0xffff0000u), zz[2 * e + 1], dacc);
+          }
+          st_shared_v4(tile + sw128_offset(r, cb), w[0], w[1], w[2], w[3]);
+        }
+      } else {
+#pragma unroll
+        for (int cb = 0; cb < 8; ++cb) st_shared_v4(tile + sw128_offset(r, cb), 0u, 0u, 0u, 0u);
+      }
+      denp[sub * 128 + r] = dacc;
+      fence_async_smem();
+    }
+    mbar_arrive(smem_u32(lsum_bar));
+    ok = ok && mbar_wait(smem_u32(lsum_bar), 0, &abort_flag, p.status);
+    ok = ok && mbar_wait(smem_u32(o_full), 0, &abort_flag, p.status);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
     const uint32_t eoff = static_cast<uint32_t>(32 * wq) << 16;
     if (ok) {
+      // O = O_s / l + O_lin / den, one rounding to bf16
       const float inv = 1.f / rowsum[r];
+      const float invd = lin ? 1.f / (denp[r] + denp[128 + r]) : 0.f;
       const size_t row = static_cast<size_t>(bh) * p.N + (row_valid ? tok : 0);
-      const __nv_bfloat16* olr = p.Ol ? p.Ol + row * kHeadDim + 64 * sub : nullptr;
       __nv_bfloat16* dst = p.out + row * kHeadDim + 64 * sub;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        uint32_t o[32];
+        uint32_t o[32], ol[32];
         tmem_ld32_sync(taddr + eoff + kColO + 64 * sub + 32 * cc, o);
+        if (lin) tmem_ld32_sync(taddr + eoff + 64 * sub + 32 * cc, ol);
         if (row_valid) {
-          float lin[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) lin[c] = 0.f;
-          if (olr) {
-            const uint4* s4 = reinterpret_cast<const uint4*>(olr + 32 * cc);
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              const uint4 u = s4[qq];
-              const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(b2[e]);
-                lin[8 * qq + 2 * e] = f.x;
-                lin[8 * qq + 2 * e + 1] = f.y;
-              }
-            }
-          }
           uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cc);
 #pragma unroll
           for (int qq = 0; qq < 4; ++qq) {
             float f[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = fmaf(__uint_as_float(o[8 * qq + e]), inv, lin[8 * qq + e]);
+            for (int e = 0; e < 8; ++e)
+              f[e] = fmaf(__uint_as_float(o[8 * qq + e]), inv, lin ? __uint_as_float(ol[8 * qq + e]) * invd : 0.f);
             d4[qq] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
                                 pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
           }
@@ -813,15 +911,17 @@ __global__ void __launch_bounds__(256) pair_kernel(const int32_t* __restrict__ c
 
 }  // namespace
 
-cudaError_t launch_attention(const Dims& g, const int8_t* q8, const int8_t* k8,
-                             const float* q_scale, const float* k_scale, const void* v,
-                             const int32_t* crit, int k_c, int m, void* out, char* ws,
+cudaError_t launch_attention(const Dims& g, const void* q, float sm_scale, const int8_t* q8,
+                             const int8_t* k8, const float* q_scale, const float* k_scale,
+                             const void* v, const int32_t* crit, int k_c, int m, void* out, char* ws,
                              cudaStream_t st) {
   const WsLayout L = ws_layout(g);
-  CUtensorMap tmQ, tmK, tmV;
+  CUtensorMap tmQ, tmK, tmV, tmH;
   if (!make_tmap_3d(&tmQ, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kHeadDim, g.Npad, g.BH, 128, 16) ||
       !make_tmap_3d(&tmK, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kHeadDim, g.Npad, g.BH, 128, 64) ||
-      !make_tmap_3d(&tmV, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim, g.N, g.BH, 64, 64))
+      !make_tmap_3d(&tmV, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim, g.N, g.BH, 64, 64) ||
+      !make_tmap_3d(&tmH, ws + L.Hbuf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim,
+                    static_cast<uint64_t>(g.nB) * kHeadDim, g.BH, 64, 64))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
   if (e != cudaSuccess) return e;
@@ -843,7 +943,10 @@ cudaError_t launch_attention(const Dims& g, const int8_t* q8, const int8_t* k8,
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.crit = crit;
-  p.Ol = m > 0 ? reinterpret_cast<const __nv_bfloat16*>(ws + L.Ol) : nullptr;
+  p.q = m > 0 ? static_cast<const __nv_bfloat16*>(q) : nullptr;
+  p.Z = reinterpret_cast<const float*>(ws + L.Zbuf);
+  p.H = reinterpret_cast<const __nv_bfloat16*>(ws + L.Hbuf);
+  p.c_s = sm_scale;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.status = reinterpret_cast<int*>(ws + L.status);
   p.N = g.N;
@@ -851,7 +954,7 @@ cudaError_t launch_attention(const Dims& g, const int8_t* q8, const int8_t* k8,
   p.k_c = k_c;
   {
     TraceScope ts_("attn_kernel", st);
-    attn_kernel<<<dim3(g.nB, g.BH), kAttnThreads, kAttnSmem, st>>>(tmQ, tmK, tmV, p);
+    attn_kernel<<<dim3(g.nB, g.BH), kAttnThreads, kAttnSmem, st>>>(tmQ, tmK, tmV, tmH, p);
   }
   return cudaGetLastError();
 }

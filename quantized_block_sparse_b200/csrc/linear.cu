@@ -16,9 +16,8 @@
 //                  hgemm_kernel's extra column tile multiplies M by [z_hi | z_lo] (exact
 //                  0/1 x bf16 products, fp32 accumulation) and Z = M.z_hi + M.z_lo in fp32,
 //                  so Z keeps about 17 significant bits of z instead of bf16's 8.
-//   linout_kernel  per pair of adjacent query blocks: phi(Q~) (recomputed from Q, bf16)
-//                  times H_i on tcgen05 (M = 128 rows = both blocks, one MMA chain per
-//                  block), divided by phi(Q~) . Z_i; bf16 O_l for the attention epilogue.
+// phi(Q~) H_i / phi(Q~) . Z_i itself is formed in the attention kernel's epilogue (the
+// H_i tiles stream through its V ring; the product lands in TMEM next to O_s).
 #include "sagesla_internal.h"
 #include "sm100_primitives.cuh"
 
@@ -222,153 +221,6 @@ __global__ void __launch_bounds__(256) zb_kernel(const float4* __restrict__ z,
   }
 }
 
-// ------------------------------------------------------------------ O_l
-// One CTA per pair of query blocks, 256 threads. Every load is issued at the start by TMA:
-// H_i0 and H_i1 (64 KB), and the pair's Q rows straight into the 128-byte-swizzled
-// K-major A tile, where phi(Q~) is computed in place (thread t: row t%128, channels
-// [64*(t/128), +64)) together with its part of the denominator. Eight warps then read the
-// two 128x128 products back (a quadrant of rows and half of the columns each), scale by
-// 1/den and stage O_l over the H tiles (swizzled) for four TMA stores.
-constexpr int kLinThreads = 256;
-constexpr int kLinSmem = 32768 + 65536 + 1024 + 1024 + 1024 + 256;
-
-__global__ void __launch_bounds__(kLinThreads) linout_kernel(const __grid_constant__ CUtensorMap tmH,
-                                                             const __grid_constant__ CUtensorMap tmQ,
-                                                             const __grid_constant__ CUtensorMap tmO,
-                                                             const float* __restrict__ Z, float c_s,
-                                                             int N, int nB, int* status) {
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  unsigned char* sA = smem;            // Q, then phi(Q~): 2 column blocks x 128 rows x 128 B
-  unsigned char* sH = smem + 32768;    // H_i0, H_i1: each 2 e-groups x 128 c rows x 128 B
-  float* dpart = reinterpret_cast<float*>(smem + 32768 + 65536);         // [2][128] denominator halves
-  float* sZ = reinterpret_cast<float*>(smem + 32768 + 65536 + 1024);     // Z_i0, Z_i1 [2][128]
-  uint64_t* lfull = reinterpret_cast<uint64_t*>(smem + 32768 + 65536 + 2048);  // Q, H, Z landed
-  uint64_t* mdone = lfull + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + 1);
-  __shared__ int abort_flag;
-
-  const int pr = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int i0 = 2 * pr;
-  const bool two = (i0 + 1) < nB;
-  if (tid == 0) {
-    abort_flag = 0;
-    mbar_init(smem_u32(lfull), 1);
-    mbar_init(smem_u32(mdone), 1);
-    fence_mbar_init();
-    mbar_expect_tx(smem_u32(lfull), (two ? 65536 + 1024 : 32768 + 512) + 32768);
-    for (int b = 0; b < (two ? 2 : 1); ++b)
-      bulk_load(smem_u32(sZ) + b * 512, Z + (static_cast<size_t>(bh) * nB + i0 + b) * kHeadDim, 512,
-                smem_u32(lfull));
-    for (int b = 0; b < (two ? 2 : 1); ++b) {
-      const uint32_t dst = smem_u32(sH) + b * 32768;
-      tma_load_3d(dst, &tmH, smem_u32(lfull), 0, (i0 + b) * 128, bh);
-      tma_load_3d(dst + 16384, &tmH, smem_u32(lfull), 64, (i0 + b) * 128, bh);
-    }
-    // Q rows of blocks i0 and i0+1 (rows past N read as zero), channel halves 0-63 / 64-127
-    for (int cb = 0; cb < 2; ++cb)
-      for (int b = 0; b < 2; ++b)
-        tma_load_3d(smem_u32(sA) + cb * 16384 + b * 8192, &tmQ, smem_u32(lfull), 64 * cb, (i0 + b) * 64, bh);
-  }
-  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 256);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t taddr = *tmem_slot;
-  bool ok = mbar_wait(smem_u32(lfull), 0, &abort_flag, status);
-  if (!ok) mbar_wait_inflight(smem_u32(lfull), 0, status);
-
-  // phi(Q~) in place for (row r, 64 channels) and that part of phi(Q~).Z_i, with the
-  // bf16-rounded phi values the tensor core sees. phi is rounded to bf16, so the fast
-  // exponential (relative error ~2^-21) is enough.
-  {
-    const int r = tid & 127, chh = tid >> 7;
-    const int i = i0 + (r >> 6);
-    const float* zr = sZ + ((i < nB) ? (r >> 6) : 0) * kHeadDim + 64 * chh;
-    const uint32_t tile = smem_u32(sA) + chh * 16384;
-    float dacc = 0.f;
-#pragma unroll
-    for (int cb = 0; cb < 8; ++cb) {  // 8 channels per 16-byte chunk
-      const uint32_t addr = tile + sw128_offset(r, cb);
-      uint32_t w[4];
-      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                   : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(addr));
-      const float4 z0 = *reinterpret_cast<const float4*>(zr + 8 * cb);
-      const float4 z1 = *reinterpret_cast<const float4*>(zr + 8 * cb + 4);
-      const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
-        const float x0 = __fmul_rn(f.x, c_s), x1 = __fmul_rn(f.y, c_s);
-        const float p0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
-        const float p1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
-        w[e] = pack_bf16x2(p0, p1);
-        const float2 pr2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
-        dacc = fmaf(pr2.x, zz[2 * e], dacc);
-        dacc = fmaf(pr2.y, zz[2 * e + 1], dacc);
-      }
-      st_shared_v4(addr, w[0], w[1], w[2], w[3]);
-    }
-    dpart[chh * 128 + r] = dacc;
-  }
-  fence_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-
-  if (tid == 0) {
-    if (ok) {
-      constexpr uint32_t idesc = make_idesc(1, 1, 0, 1, 128, 128);
-      for (int b = 0; b < (two ? 2 : 1); ++b) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = make_sdesc(smem_u32(sA) + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = make_sdesc(smem_u32(sH) + b * 32768 + kk * 2048, 16384, 1024);
-          mma_bf16(taddr + 128 * b, a, bd, idesc, kk > 0);
-        }
-      }
-    }
-    mma_commit(smem_u32(mdone));
-  }
-  __syncwarp();
-  ok = mbar_wait(smem_u32(mdone), 0, &abort_flag, status) && ok;
-  tc_fence_after();
-  // Warp w: TMEM lane quadrant w%4 (rows 32*(w%4) ..), output columns [64*(w/4), +64).
-  // Rows 0-63 (block i0) read the product with H_i0 (columns 0-127), rows 64-127 the one
-  // with H_i0+1 (columns 128-255). O_l is staged over the H tiles (free once the MMAs
-  // are done): column half ch2 at sH + 16 KB * ch2, 128 rows x 128 B, swizzled.
-  const int wq = warp & 3, ch2 = warp >> 2;
-  const int r = 32 * wq + lane;
-  const int half = wq >> 1;
-  if (ok && (i0 + half < nB)) {  // warp-uniform
-    const float inv = 1.f / (dpart[r] + dpart[128 + r]);
-    const uint32_t tile = smem_u32(sH) + ch2 * 16384;
-#pragma unroll
-    for (int cchunk = 0; cchunk < 2; ++cchunk) {
-      uint32_t rr[32];
-      tmem_ld32_sync(taddr + (static_cast<uint32_t>(32 * wq) << 16) + 128 * half + 64 * ch2 + 32 * cchunk, rr);
-#pragma unroll
-      for (int qq = 0; qq < 4; ++qq)
-        st_shared_v4(tile + sw128_offset(r, 4 * cchunk + qq),
-                     pack_bf16x2(__uint_as_float(rr[8 * qq]) * inv, __uint_as_float(rr[8 * qq + 1]) * inv),
-                     pack_bf16x2(__uint_as_float(rr[8 * qq + 2]) * inv, __uint_as_float(rr[8 * qq + 3]) * inv),
-                     pack_bf16x2(__uint_as_float(rr[8 * qq + 4]) * inv, __uint_as_float(rr[8 * qq + 5]) * inv),
-                     pack_bf16x2(__uint_as_float(rr[8 * qq + 6]) * inv, __uint_as_float(rr[8 * qq + 7]) * inv));
-    }
-    fence_async_smem();
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(taddr, 256);
-  if (tid == 0 && ok) {  // rows past N fall outside the tensor and are not written
-    for (int b = 0; b < (two ? 2 : 1); ++b)
-      for (int cb = 0; cb < 2; ++cb)
-        tma_store_3d(&tmO, smem_u32(sH) + cb * 16384 + b * 8192, 64 * cb, (i0 + b) * 64, bh);
-    bulk_store_commit_wait_read();
-  }
-}
-
 }  // namespace
 
 // Sums of per-key-block states over a 0/1 block mask, per head: Hout[i] = sum_j M[i][j] h[j]
@@ -405,33 +257,13 @@ cudaError_t launch_mask_gemm(const Dims& g, const void* mask, const void* h, con
   return cudaGetLastError();
 }
 
-cudaError_t launch_linear(const Dims& g, const void* q, float sm_scale, const void* mask,
-                          const int32_t* marg, int m, const void* h, const float* z, char* ws,
-                          cudaStream_t st) {
+cudaError_t launch_linear(const Dims& g, const void* mask, int m, const void* h, const float* z,
+                          char* ws, cudaStream_t st) {
   if (m == 0) return cudaSuccess;
   const WsLayout L = ws_layout(g);
-  int* status = reinterpret_cast<int*>(ws + L.status);
-  __nv_bfloat16* Hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.Hbuf);
-  float* Zbuf = reinterpret_cast<float*>(ws + L.Zbuf);
-  __nv_bfloat16* Ol = reinterpret_cast<__nv_bfloat16*>(ws + L.Ol);
-  __nv_bfloat16* Zb = reinterpret_cast<__nv_bfloat16*>(ws + L.Zb);
-
-  cudaError_t e = launch_mask_gemm(g, mask, h, z, Hbuf, Zbuf, Zb, status, st);
-  if (e != cudaSuccess) return e;
-  CUtensorMap tmH, tmQ, tmO;
-  if (!make_tmap_3d(&tmH, Hbuf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim,
-                    static_cast<uint64_t>(g.nB) * kHeadDim, g.BH, 64, 128) ||
-      !make_tmap_3d(&tmQ, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim, g.N, g.BH, 64, 64) ||
-      !make_tmap_3d(&tmO, Ol, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kHeadDim, g.N, g.BH, 64, 64))
-    return cudaErrorInvalidValue;
-  e = cudaFuncSetAttribute(linout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem);
-  if (e != cudaSuccess) return e;
-  {
-    TraceScope ts_("linout_kernel", st);
-    linout_kernel<<<dim3((g.nB + 1) / 2, g.BH), kLinThreads, kLinSmem, st>>>(tmH, tmQ, tmO, Zbuf, sm_scale,
-                                                                          g.N, g.nB, status);
-  }
-  return cudaGetLastError();
+  return launch_mask_gemm(g, mask, h, z, reinterpret_cast<__nv_bfloat16*>(ws + L.Hbuf),
+                          reinterpret_cast<float*>(ws + L.Zbuf), reinterpret_cast<__nv_bfloat16*>(ws + L.Zb),
+                          reinterpret_cast<int*>(ws + L.status), st);
 }
 
 }  // namespace sgs

@@ -30,7 +30,6 @@ struct WsLayout {
   size_t Zb;         // bf16 [BH, nB, 2d]     [z_hi | z_lo], z split into two bf16 parts
   size_t pairs;      // int2 [BH, nB]         query-block pairs of the attention tiles
   size_t pair_counts;  // int32 [BH, ceil(nB/64)] tiles per pairing segment
-  size_t Ol;         // bf16 [BH, N, d]
   size_t total;
 };
 WsLayout ws_layout(const Dims& g);
@@ -45,16 +44,19 @@ cudaError_t launch_select(const Dims& g, const float* q_bar, const float* k_bar,
                           int n_neg, int m, int32_t* crit, int32_t* marg, void* mask,
                           float* logits, cudaStream_t st);
 // linear.cu
-cudaError_t launch_linear(const Dims& g, const void* q, float sm_scale, const void* mask,
-                          const int32_t* marg, int m, const void* h, const float* z, char* ws,
-                          cudaStream_t st);
+// H_i = sum of h_j and Z_i = sum of z_j over the marginal blocks of i, into the workspace
+// (nothing when m == 0).
+cudaError_t launch_linear(const Dims& g, const void* mask, int m, const void* h, const float* z,
+                          char* ws, cudaStream_t st);
 cudaError_t launch_mask_gemm(const Dims& g, const void* mask, const void* h, const float* z,
                              __nv_bfloat16* Hout, float* Zout, __nv_bfloat16* zb, int* status,
                              cudaStream_t st);
 // attention.cu
-cudaError_t launch_attention(const Dims& g, const int8_t* q8, const int8_t* k8,
-                             const float* q_scale, const float* k_scale, const void* v,
-                             const int32_t* crit, int k_c, int m, void* out, char* ws,
+// Critical-block attention, plus (m > 0) the linear term from the workspace's H_i, Z_i and
+// phi(Q*sm_scale) recomputed from q; out = O_s + O_l in bf16.
+cudaError_t launch_attention(const Dims& g, const void* q, float sm_scale, const int8_t* q8,
+                             const int8_t* k8, const float* q_scale, const float* k_scale,
+                             const void* v, const int32_t* crit, int k_c, int m, void* out, char* ws,
                              cudaStream_t st);
 
 // backward.cu

@@ -53,7 +53,7 @@ def test_counts_match_oracle(L, N, rho, nu):
 def test_workspace_bytes(L):
     n = S.sagesla_workspace_bytes(1, 12, 32760)
     nB = 512
-    assert n >= 12 * nB * 128 * 128 * 2 + 12 * 32760 * 128 * 2
+    assert n >= 12 * nB * 128 * 128 * 2  # H, bf16
     with pytest.raises(S.SageSLAError):
         S.sagesla_workspace_bytes(1, 12, 32760, d=64)
 
