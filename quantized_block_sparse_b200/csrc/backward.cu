@@ -18,6 +18,8 @@
 //
 // Kernels (bf16 operands, fp32 accumulation on the mma.sync m16n8k16 tensor-core path;
 // 64-token blocks, four warps of 16 rows each):
+//   tilde_kernel   Q~ and K~ rounded to bf16 once, so that the loops below stream raw tiles
+//                  (cp.async into two buffers: the next tile's copy overlaps this one's math).
 //   bwd_q_kernel   per query block: a statistics pass over the critical blocks (online
 //                  softmax: O_s, LSE, D), a dQ pass, and the linear branch's dQ, dH_i, dZ_i.
 //   (mask GEMM)    H = M h, Z = M z before, and G = M^T dH, g = M^T dZ after bwd_q_kernel
@@ -37,12 +39,16 @@ namespace bwd {
 constexpr int kLd = 136;                 // shared row stride in bf16 elements (272 B, conflict-free)
 constexpr int kTileElems = 64 * kLd;     // one 64 x 128 tile
 constexpr int kThreads = 128;
-constexpr int kQSmem = (4 * kTileElems + 128 * kLd) * 2 + (64 + 64 + 128 + 64) * 4;
-constexpr int kKVSmem = (4 * kTileElems + 128 * kLd) * 2 + (64 + 64 + 128) * 4;
+// Six 64 x 128 tiles: two fixed ones and two double-buffered pairs (the last pair of tiles
+// also holds the 128-row H_i or G_j of the linear branch once the loops are done).
+constexpr int kQSmem = 6 * kTileElems * 2 + (64 + 64 + 128 + 64) * 4;
+constexpr int kKVSmem = 6 * kTileElems * 2 + (2 * 64 + 2 * 64 + 128) * 4;
 
 struct Params {
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
+  const __nv_bfloat16* qt;  // bf16(fl32(Q c_s)), [BH, N, d]
+  const __nv_bfloat16* kt;  // bf16(fl32(K - mu)), [BH, N, d]
   const __nv_bfloat16* v;
   const __nv_bfloat16* dout;
   const float* k_mean;
@@ -156,6 +162,28 @@ __device__ __forceinline__ void load_tile(__nv_bfloat16* dst, const __nv_bfloat1
   }
 }
 
+// ---- asynchronous tile copies (cp.async, 16 B per thread; a zero-byte source fills zeros)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
+// Rows [64*blk, 64*blk + 64) of one head's [N, 128] bf16 tensor, as stored, into a padded
+// shared tile; rows past N are zero.
+__device__ __forceinline__ void issue_tile(uint32_t dst, const __nv_bfloat16* src, int blk, int N) {
+  for (int x = threadIdx.x; x < 64 * 16; x += blockDim.x) {
+    const int r = x >> 4, c8 = (x & 15) * 8;
+    const int tok = blk * 64 + r;
+    const bool in = tok < N;
+    cp_async16(dst + static_cast<uint32_t>((r * kLd + c8) * 2),
+               src + static_cast<size_t>(in ? tok : 0) * kHeadDim + c8, in ? 16u : 0u);
+  }
+}
+
 __device__ __forceinline__ float quad_sum(float v) {
   v += __shfl_xor_sync(0xffffffffu, v, 1);
   return v + __shfl_xor_sync(0xffffffffu, v, 2);
@@ -205,9 +233,9 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(Params p) {
   extern __shared__ __align__(16) unsigned char sm[];
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(sm);  // Q~ of block i
   __nv_bfloat16* sO = sQ + kTileElems;                        // dO of block i
-  __nv_bfloat16* sK = sO + kTileElems;                        // K~_j, later phi(Q~)
-  __nv_bfloat16* sV = sK + kTileElems;                        // V_j, later dn
-  __nv_bfloat16* sH = sV + kTileElems;                        // H_i [128][kLd]
+  __nv_bfloat16* sK = sO + kTileElems;                        // K~_j / V_j buffer 0, later phi(Q~)
+  __nv_bfloat16* sV = sK + kTileElems;                        //   and dn
+  __nv_bfloat16* sH = sV + kTileElems;                        // K~_j / V_j buffer 1, later H_i [128][kLd]
   float* sDen = reinterpret_cast<float*>(sH + 128 * kLd);     // [64]
   float* sDd = sDen + 64;                                     // dden [64]
   float* sZ = sDd + 64;                                       // Z_i [128]
@@ -219,10 +247,20 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(Params p) {
   const float* mu = p.k_mean + static_cast<size_t>(bh) * kHeadDim;
   const uint32_t aQ = smem_u32(sQ), aO = smem_u32(sO), aK = smem_u32(sK), aV = smem_u32(sV),
                  aH = smem_u32(sH);
-  load_tile<1>(sQ, p.q + head, i, p.N, p.c_s, mu);
-  load_tile<0>(sO, p.dout + head, i, p.N, p.c_s, mu);
   const int32_t* crit = p.crit + (static_cast<size_t>(bh) * p.nB + i) * p.k_c;
   const int rowA = i * 64 + r0 + g, rowB = rowA + 8;  // this thread's two query rows
+  // K~_j and V_j of the walk's step jj go to buffer jj & 1 (tiles 2-3 or 4-5); the copies
+  // of step jj + 1 run while step jj computes.
+  auto issue_kv = [&](int jj) {
+    const int j = __ldg(crit + jj);
+    const uint32_t base = aK + static_cast<uint32_t>((jj & 1) * 2 * kTileElems * 2);
+    issue_tile(base, p.kt + head, j, p.N);
+    issue_tile(base + kTileElems * 2, p.v + head, j, p.N);
+    cp_async_commit();
+  };
+  issue_tile(aQ, p.qt + head, i, p.N);
+  issue_tile(aO, p.dout + head, i, p.N);
+  issue_kv(0);  // one group with Q~ and dO
 
   // ---- pass 1: online softmax over the critical blocks -> O_s, LSE, D
   float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
@@ -231,12 +269,16 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(Params p) {
   for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
   for (int jj = 0; jj < p.k_c; ++jj) {
     const int j = __ldg(crit + jj);
+    if (jj + 1 < p.k_c) {
+      issue_kv(jj + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
     __syncthreads();
-    load_tile<2>(sK, p.k + head, j, p.N, p.c_s, mu);
-    load_tile<0>(sV, p.v + head, j, p.N, p.c_s, mu);
-    __syncthreads();
+    const uint32_t aKj = aK + static_cast<uint32_t>((jj & 1) * 2 * kTileElems * 2), aVj = aKj + kTileElems * 2;
     float s[8][4];
-    gemm_16x64_k128(s, aQ, r0, aK, lane);
+    gemm_16x64_k128(s, aQ, r0, aKj, lane);
     const int nvalid = min(64, p.N - j * 64);
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
@@ -266,7 +308,8 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(Params p) {
         o[nt][2 * h + 1] *= alpha;
       }
     }
-    gemm_acc_16x128_k64(o, s, aV, lane);
+    gemm_acc_16x128_k64(o, s, aVj, lane);
+    __syncthreads();  // buffer jj & 1 is free for step jj + 2
   }
   float lse[2], dd[2];
 #pragma unroll
@@ -295,15 +338,20 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(Params p) {
   float dq[16][4];
 #pragma unroll
   for (int nt = 0; nt < 16; ++nt) dq[nt][0] = dq[nt][1] = dq[nt][2] = dq[nt][3] = 0.f;
+  issue_kv(0);
   for (int jj = 0; jj < p.k_c; ++jj) {
     const int j = __ldg(crit + jj);
+    if (jj + 1 < p.k_c) {
+      issue_kv(jj + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
     __syncthreads();
-    load_tile<2>(sK, p.k + head, j, p.N, p.c_s, mu);
-    load_tile<0>(sV, p.v + head, j, p.N, p.c_s, mu);
-    __syncthreads();
+    const uint32_t aKj = aK + static_cast<uint32_t>((jj & 1) * 2 * kTileElems * 2), aVj = aKj + kTileElems * 2;
     float s[8][4], dp[8][4];
-    gemm_16x64_k128(s, aQ, r0, aK, lane);
-    gemm_16x64_k128(dp, aO, r0, aV, lane);
+    gemm_16x64_k128(s, aQ, r0, aKj, lane);
+    gemm_16x64_k128(dp, aO, r0, aVj, lane);
     const int nvalid = min(64, p.N - j * 64);
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
@@ -313,7 +361,8 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(Params p) {
         const float pr = (8 * nt + 2 * t4 + (e & 1) < nvalid) ? __expf(s[nt][e] - lse[h]) : 0.f;
         s[nt][e] = pr * (dp[nt][e] - dd[h]);  // dS
       }
-    gemm_acc_16x128_k64(dq, s, aK, lane);
+    gemm_acc_16x128_k64(dq, s, aKj, lane);
+    __syncthreads();  // buffer jj & 1 is free for step jj + 2
   }
 
   // ---- linear branch: dQ~ += dphi o phi'(Q~); dH_i, dZ_i
@@ -473,58 +522,89 @@ __global__ void __launch_bounds__(kThreads) bwd_kv_kernel(Params p) {
   extern __shared__ __align__(16) unsigned char sm[];
   __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(sm);  // K~_j
   __nv_bfloat16* sV = sK + kTileElems;                        // V_j
-  __nv_bfloat16* sQ = sV + kTileElems;                        // Q~_i, later phi(K~_j)
-  __nv_bfloat16* sO = sQ + kTileElems;                        // dO_i
-  __nv_bfloat16* sG = sO + kTileElems;                        // G_j [128][kLd]
-  float* sL = reinterpret_cast<float*>(sG + 128 * kLd);       // LSE_i [64]
-  float* sD = sL + 64;                                        // D_i [64]
-  float* sg = sD + 64;                                        // g_j [128]
+  __nv_bfloat16* sQ = sV + kTileElems;                        // Q~_i / dO_i buffer 0, later phi(K~_j)
+  __nv_bfloat16* sG = sQ + 2 * kTileElems;                    // Q~_i / dO_i buffer 1, later G_j [128][kLd]
+  float* sLD = reinterpret_cast<float*>(sm + 6 * kTileElems * 2);  // [2 buffers][LSE_i 64 | D_i 64]
+  float* sg = sLD + 2 * 128;                                        // g_j [128]
   const int j = blockIdx.x, bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
   const int r0 = 16 * warp;
   const size_t head = static_cast<size_t>(bh) * p.N * kHeadDim;
   const float* mu = p.k_mean + static_cast<size_t>(bh) * kHeadDim;
-  const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aO = smem_u32(sO),
-                 aG = smem_u32(sG);
-  load_tile<2>(sK, p.k + head, j, p.N, p.c_s, mu);
-  load_tile<0>(sV, p.v + head, j, p.N, p.c_s, mu);
+  const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aG = smem_u32(sG),
+                 aLD = smem_u32(sLD);
+  // Q~_i, dO_i, LSE_i and D_i of the n-th query block of the walk go to buffer n & 1; the
+  // copies of the next block run while this one computes.
+  auto issue_q = [&](int i, int buf) {
+    const uint32_t base = aQ + static_cast<uint32_t>(buf * 2 * kTileElems * 2);
+    issue_tile(base, p.qt + head, i, p.N);
+    issue_tile(base + kTileElems * 2, p.dout + head, i, p.N);
+    if (threadIdx.x < 32) {  // 2 x 256 B
+      const size_t off = static_cast<size_t>(bh) * p.Npad + i * 64 + 4 * (threadIdx.x & 15);
+      cp_async16(aLD + static_cast<uint32_t>((buf * 128 + 64 * (threadIdx.x >> 4) + 4 * (threadIdx.x & 15)) * 4),
+                 ((threadIdx.x >> 4) ? p.dd : p.lse) + off, 16u);
+    }
+    cp_async_commit();
+  };
+  // the query blocks holding j critical, in increasing order (bits of cbits[bh][j])
+  const uint32_t* bits = p.cbits + (static_cast<size_t>(bh) * p.nB + j) * p.nW;
+  int w = 0;
+  uint32_t word = p.nW > 0 ? __ldg(bits) : 0u;
+  auto next_i = [&]() -> int {
+    while (word == 0u) {
+      if (++w >= p.nW) return -1;
+      word = __ldg(bits + w);
+    }
+    const int i = 32 * w + __ffs(word) - 1;
+    word &= word - 1;
+    return i;
+  };
+  issue_tile(aK, p.kt + head, j, p.N);
+  issue_tile(aV, p.v + head, j, p.N);
+  int i_cur = next_i();
+  if (i_cur >= 0) {
+    issue_q(i_cur, 0);  // one group with K~_j and V_j
+  } else {
+    cp_async_commit();
+  }
   float dk[16][4], dv[16][4];
 #pragma unroll
   for (int nt = 0; nt < 16; ++nt) {
     dk[nt][0] = dk[nt][1] = dk[nt][2] = dk[nt][3] = 0.f;
     dv[nt][0] = dv[nt][1] = dv[nt][2] = dv[nt][3] = 0.f;
   }
-  const uint32_t* bits = p.cbits + (static_cast<size_t>(bh) * p.nB + j) * p.nW;
-  for (int w = 0; w < p.nW; ++w) {
-    uint32_t word = __ldg(bits + w);
-    while (word) {
-      const int i = 32 * w + __ffs(word) - 1;
-      word &= word - 1;
-      __syncthreads();
-      load_tile<1>(sQ, p.q + head, i, p.N, p.c_s, mu);
-      load_tile<0>(sO, p.dout + head, i, p.N, p.c_s, mu);
-      if (threadIdx.x < 64) {
-        sL[threadIdx.x] = p.lse[static_cast<size_t>(bh) * p.Npad + i * 64 + threadIdx.x];
-        sD[threadIdx.x] = p.dd[static_cast<size_t>(bh) * p.Npad + i * 64 + threadIdx.x];
-      }
-      __syncthreads();
-      float st[8][4], dpt[8][4];
-      gemm_16x64_k128(st, aK, r0, aQ, lane);   // S^T: keys x queries
-      gemm_16x64_k128(dpt, aV, r0, aO, lane);  // dP^T = V dO^T
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int qc = 8 * nt + 2 * t4 + (e & 1);
-          st[nt][e] = __expf(st[nt][e] - sL[qc]);           // P^T (0 for query rows past N)
-          dpt[nt][e] = st[nt][e] * (dpt[nt][e] - sD[qc]);  // dS^T
-        }
-      gemm_acc_16x128_k64(dv, st, aO, lane);   // dV += P^T dO
-      gemm_acc_16x128_k64(dk, dpt, aQ, lane);  // dK~ += dS^T Q~
+  for (int n = 0; i_cur >= 0; ++n) {
+    const int i_nxt = next_i();
+    if (i_nxt >= 0) {
+      issue_q(i_nxt, (n + 1) & 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-  }
-  if (p.m > 0) {
     __syncthreads();
+    const int b = n & 1;
+    const uint32_t aQi = aQ + static_cast<uint32_t>(b * 2 * kTileElems * 2), aOi = aQi + kTileElems * 2;
+    const float* sL = sLD + b * 128;
+    const float* sD = sL + 64;
+    float st[8][4], dpt[8][4];
+    gemm_16x64_k128(st, aK, r0, aQi, lane);   // S^T: keys x queries
+    gemm_16x64_k128(dpt, aV, r0, aOi, lane);  // dP^T = V dO^T
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int qc = 8 * nt + 2 * t4 + (e & 1);
+        st[nt][e] = __expf(st[nt][e] - sL[qc]);           // P^T (0 for query rows past N)
+        dpt[nt][e] = st[nt][e] * (dpt[nt][e] - sD[qc]);  // dS^T
+      }
+    gemm_acc_16x128_k64(dv, st, aOi, lane);   // dV += P^T dO
+    gemm_acc_16x128_k64(dk, dpt, aQi, lane);  // dK~ += dS^T Q~
+    __syncthreads();  // buffer n & 1 is free for block n + 2
+    i_cur = i_nxt;
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  if (p.m > 0) {
     load_tile<4>(sQ, p.k + head, j, p.N, p.c_s, mu);  // phi(K~_j), zero rows past N
     const __nv_bfloat16* Gj = p.G + (static_cast<size_t>(bh) * p.nB + j) * kHeadDim * kHeadDim;
     for (int x = threadIdx.x; x < 128 * 16; x += blockDim.x) {
@@ -602,6 +682,31 @@ __global__ void __launch_bounds__(kThreads) bwd_kv_kernel(Params p) {
   }
 }
 
+// Q~ = bf16(fl32(Q c_s)) and K~ = bf16(fl32(K - mu)), the operand tiles the two kernels
+// stream (the same roundings a tile loader applying them on the fly would make).
+__global__ void __launch_bounds__(256) tilde_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
+                                                    const float* __restrict__ k_mean, float c_s,
+                                                    uint4* __restrict__ qt, uint4* __restrict__ kt,
+                                                    size_t n8, int N) {
+  for (size_t x = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; x < n8;
+       x += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t bh = x / (static_cast<size_t>(N) * 16);
+    const int c8 = static_cast<int>(x % 16) * 8;
+    const float* mu = k_mean + bh * kHeadDim + c8;
+    const uint4 uq = q[x], uk = k[x];
+    uint32_t wq[4] = {uq.x, uq.y, uq.z, uq.w}, wk[4] = {uk.x, uk.y, uk.z, uk.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 fq = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wq[e]));
+      const float2 fk = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wk[e]));
+      wq[e] = pack_bf16x2(__fmul_rn(fq.x, c_s), __fmul_rn(fq.y, c_s));
+      wk[e] = pack_bf16x2(__fsub_rn(fk.x, mu[2 * e]), __fsub_rn(fk.y, mu[2 * e + 1]));
+    }
+    qt[x] = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+    kt[x] = make_uint4(wk[0], wk[1], wk[2], wk[3]);
+  }
+}
+
 // Key block j is critical for query block i: bit i of cbits[bh][j].
 __global__ void __launch_bounds__(64) crit_bits_kernel(const int32_t* __restrict__ crit, int nB, int k_c,
                                                        int nW, uint32_t* __restrict__ cbits) {
@@ -660,7 +765,7 @@ __global__ void __launch_bounds__(256) dk_sub_kernel(float4* __restrict__ dk, co
 
 // Workspace of the backward pass (byte offsets, 256-aligned).
 struct BwdLayout {
-  size_t status, H, Z, zb, lse, dd, dH, dZ, G, gz, maskT, cbits, kpart, kmean, total;
+  size_t status, H, Z, zb, lse, dd, dH, dZ, G, gz, maskT, cbits, kpart, kmean, qt, kt, total;
   int nW;
 };
 static size_t a256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -688,6 +793,8 @@ BwdLayout bwd_layout(const Dims& g) {
   L.cbits = take(BH * nB * L.nW * 4);
   L.kpart = take(BH * nB * kHeadDim * 4);
   L.kmean = take(BH * kHeadDim * 4);
+  L.qt = take(BH * g.N * kHeadDim * 2);
+  L.kt = take(BH * g.N * kHeadDim * 2);
   L.total = off;
   return L;
 }
@@ -703,6 +810,8 @@ cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const v
   bwd::Params p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k = static_cast<const __nv_bfloat16*>(k);
+  p.qt = reinterpret_cast<const __nv_bfloat16*>(ws + L.qt);
+  p.kt = reinterpret_cast<const __nv_bfloat16*>(ws + L.kt);
   p.v = static_cast<const __nv_bfloat16*>(v);
   p.dout = static_cast<const __nv_bfloat16*>(dout);
   p.k_mean = k_mean;
@@ -733,6 +842,14 @@ cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const v
     e = launch_mask_gemm(g, mask, h, z, reinterpret_cast<__nv_bfloat16*>(ws + L.H),
                          reinterpret_cast<float*>(ws + L.Z), zb, status, st);
     if (e != cudaSuccess) return e;
+  }
+  {
+    TraceScope ts_("tilde_kernel", st);
+    const size_t n8 = static_cast<size_t>(g.BH) * g.N * 16;
+    const int blocks = static_cast<int>((n8 + 255) / 256 < 8192 ? (n8 + 255) / 256 : 8192);
+    bwd::tilde_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint4*>(q), static_cast<const uint4*>(k), k_mean,
+                                              sm_scale, reinterpret_cast<uint4*>(ws + L.qt),
+                                              reinterpret_cast<uint4*>(ws + L.kt), n8, g.N);
   }
   e = cudaFuncSetAttribute(bwd::bwd_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::kQSmem);
   if (e != cudaSuccess) return e;
