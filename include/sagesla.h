@@ -152,6 +152,21 @@ int sagesla_forward(const sagesla_shape* shape, const void* q, float sm_scale,
                     const float* z, void* out, void* workspace, size_t workspace_bytes,
                     void* stream);
 
+/* Step (6), first half, on its own (the GEMM sagesla_forward runs before its attention):
+ * H_i = sum of h_j and Z_i = sum of z_j over the marginal key blocks j of query block i
+ * ("TurboDiffusion Demystified", section "Pillar Two: Sparse-Linear Attention - SLA": the
+ * linear term covers the marginal blocks), as one GEMM with the 0/1 mask.
+ * Inputs : marg_mask bf16 [B,H,nB,nBp] and m from sagesla_select; h bf16 [B,H,nB,d,d] and
+ *          z fp32 [B,H,nB,d] from sagesla_prepare. 0 <= m <= nB - 1.
+ * Outputs: H bf16 [B,H,nB,d,d]: fp32 tensor-core sums of the exact 0/1 x bf16 products,
+ *          rounded once (RNE). Z fp32 [B,H,nB,d]: z split into z_hi = bf16(z) and
+ *          z_lo = bf16(z - z_hi), each summed in fp32, the two sums added.
+ * workspace: at least sagesla_workspace_bytes(shape) bytes (the bf16 split of z and the
+ *          status word live there). A row with no marginal block gets H_i = 0, Z_i = 0. */
+int sagesla_marginal_sums(const sagesla_shape* shape, const void* marg_mask, int m,
+                          const void* h, const float* z, void* H, float* Z, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
 /* Synchronize `stream`, then return the workspace status word: SAGESLA_OK, or
  * SAGESLA_ERR_TIMEOUT if a bounded device wait gave up (the affected output is
  * invalid), or SAGESLA_ERR_CUDA if the stream reported an error. */

@@ -256,6 +256,25 @@ int sagesla_forward(const sagesla_shape* shape, const void* q, float sm_scale, c
                                          out, ws, st));
 }
 
+int sagesla_marginal_sums(const sagesla_shape* shape, const void* marg_mask, int m, const void* h,
+                          const float* z, void* H, float* Z, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  Dims g;
+  int rc = make_dims(shape, &g);
+  if (rc != SAGESLA_OK) return rc;
+  if (m < 0 || m > g.nB - 1) return SAGESLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {marg_mask, h, z, H, Z, workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return SAGESLA_ERR_INVALID_ARG;
+  const sgs::WsLayout L = sgs::ws_layout(g);
+  if (workspace_bytes < L.total) return SAGESLA_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  return from_cuda(sgs::launch_mask_gemm(g, marg_mask, h, z, static_cast<__nv_bfloat16*>(H), Z,
+                                         reinterpret_cast<__nv_bfloat16*>(ws + L.Zb),
+                                         reinterpret_cast<int*>(ws + L.status),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 size_t sagesla_backward_workspace_bytes(const sagesla_shape* shape) {
   Dims g;
   if (make_dims(shape, &g) != SAGESLA_OK) return 0;

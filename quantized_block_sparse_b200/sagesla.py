@@ -76,6 +76,8 @@ def lib():
     L.sagesla_forward.argtypes = ([sp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int,
                                    _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp])
     L.sagesla_forward.restype = ctypes.c_int
+    L.sagesla_marginal_sums.argtypes = [sp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    L.sagesla_marginal_sums.restype = ctypes.c_int
     L.sagesla_check_status.argtypes = [_vp, _vp]
     L.sagesla_check_status.restype = ctypes.c_int
     L.sagesla_status_string.argtypes = [ctypes.c_int]
@@ -244,6 +246,21 @@ def sagesla_forward(q, v, prep: Prepared, sel: Selection, workspace, out=None, s
                                  _ptr(prep.z), _ptr(out), _ptr(workspace), workspace.numel(),
                                  _stream(stream)), "sagesla_forward")
     return out
+
+
+def sagesla_marginal_sums(mask, m, h, z, workspace, N=None, stream=None):
+    """H_i = sum of h_j, Z_i = sum of z_j over the marginal blocks of each query block (the
+    first half of step 6 on its own). mask bf16 [B,H,nB,nBp], h bf16 [B,H,nB,128,128],
+    z fp32 [B,H,nB,128], N the token count (default 64 nB) -> (H bf16 like h, Z fp32 like z)."""
+    B, H, nB = h.shape[:3]
+    N = 64 * nB if N is None else int(N)
+    assert h.dtype == torch.bfloat16 and z.dtype == torch.float32 and mask.dtype == torch.bfloat16
+    Hout = torch.empty_like(h)
+    Zout = torch.empty_like(z)
+    _check(lib().sagesla_marginal_sums(ctypes.byref(_shape(B, H, N, HEAD_DIM)), _ptr(mask), int(m), _ptr(h),
+                                       _ptr(z), _ptr(Hout), _ptr(Zout), _ptr(workspace), workspace.numel(),
+                                       _stream(stream)), "sagesla_marginal_sums")
+    return Hout, Zout
 
 
 def sagesla_check_status(workspace, stream=None):

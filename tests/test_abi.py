@@ -133,6 +133,14 @@ def test_more_validation_paths(L):
     assert L.sagesla_selftest_wait_timeout(p, 128, 1000, None) == 1
     assert L.sagesla_selftest_wait_timeout(p, 1 << 20, 0, None) == 1
     assert L.sagesla_selftest_wait_timeout(p, 1 << 20, 1000001, None) == 1
+    # the marginal sums on their own: m in 0..nB-1, aligned pointers, a large enough workspace
+    # (shape N = 1024: nB = 16)
+    assert L.sagesla_marginal_sums(ctypes.byref(sh), p, -1, p, p, p, p, p, big, None) == 1
+    assert L.sagesla_marginal_sums(ctypes.byref(sh), p, 16, p, p, p, p, p, big, None) == 1
+    assert L.sagesla_marginal_sums(ctypes.byref(sh), p, 4, p, mis, p, p, p, big, None) == 1
+    assert L.sagesla_marginal_sums(ctypes.byref(sh), p, 4, p, p, None, p, p, big, None) == 1
+    assert L.sagesla_marginal_sums(ctypes.byref(sh), p, 4, p, p, p, p, p, 256, None) == 1
+    assert L.sagesla_marginal_sums(ctypes.byref(_sh(d=64)), p, 4, p, p, p, p, p, big, None) == 2
 
 
 def test_status_strings(L):
