@@ -32,6 +32,9 @@ WsLayout ws_layout(const Dims& g) {
   off = align256(off + static_cast<size_t>(g.BH) * g.nB * 8);
   L.pair_counts = off;
   off = align256(off + static_cast<size_t>(g.BH) * ((g.nB + 63) / 64) * 4);
+  const bool whole = whole_head_pairing(g);
+  L.pair_window = off;
+  off = align256(off + (whole ? static_cast<size_t>(g.BH) * g.nB * 128 : 0));
   L.total = off;
   return L;
 }

@@ -30,9 +30,17 @@ struct WsLayout {
   size_t Zb;         // bf16 [BH, nB, 2d]     [z_hi | z_lo], z split into two bf16 parts
   size_t pairs;      // int2 [BH, nB]         query-block pairs of the attention tiles
   size_t pair_counts;  // int32 [BH, ceil(nB/64)] tiles per pairing segment
+  size_t pair_window;  // uint8 [BH, nB, 128] critical-set overlaps with the next 127 blocks
   size_t total;
 };
 WsLayout ws_layout(const Dims& g);
+// Whole-head pairing of query blocks (one warp scans a head's blocks in order, its window
+// table in shared memory) for heads of 769 to 1664 blocks with at most 256 MiB of tables; for
+// shorter heads the sequential scan costs more than the union steps it saves, and longer ones
+// do not fit. Otherwise pairs are chosen within segments of 64 blocks.
+inline bool whole_head_pairing(const Dims& g) {
+  return g.nB > 768 && g.nB <= 1664 && static_cast<size_t>(g.BH) * g.nB * 128 <= (static_cast<size_t>(256) << 20);
+}
 
 // prepare.cu
 cudaError_t launch_prepare(const Dims& g, const void* q, const void* k, const void* v,

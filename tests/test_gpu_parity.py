@@ -195,3 +195,32 @@ def test_select_at_the_block_limit():
     np.put_along_axis(member, marg.astype(np.int64), 2, axis=1)
     assert ((member == 1).sum(1) == sel.k_c).all() and ((member == 2).sum(1) == sel.m).all()
     np.testing.assert_array_equal(mask[:, :8192], (member == 2).astype(np.float32))
+
+
+def test_whole_head_pairing_writes_every_row():
+    # 800 blocks per head take the whole-head pairing of query blocks (a sequential greedy
+    # over the head); a block missing from the tile list would leave its rows unwritten, so
+    # the output starts as NaN and every real row must be finite afterwards. Sampled query
+    # blocks of the first head are then checked against the oracle.
+    import torch
+    from quantized_block_sparse_b200 import sagesla as S
+    from tests.gpu_helpers import ensure_lib
+    ensure_lib()
+    B, H, grid, rho, nu = 1, 2, (10, 40, 128), 0.1, 0.45  # N = 51200: nB = 800
+    q, k, v = make_qkv(B, H, grid, seed=3)
+    N = q.shape[2]
+    eng = S.SageSLA(B, H, N, rho, nu)
+    eng.out.fill_(float("nan"))
+    out = eng(q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    eng.check()
+    o = out.float().cpu().numpy()
+    assert np.isfinite(o).all()
+    qf, kf, vf = f32(q[:, :1]), f32(k[:, :1]), f32(v[:, :1])
+    prep = O.prepare(qf, kf)
+    sel = O.select(prep.q_bar, prep.k_bar, rho, nu)
+    rng = np.random.default_rng(11)
+    qb = sorted(set(rng.choice(800, size=10, replace=False).tolist()) | {0, 799})
+    ref = O.forward(prep, vf, sel, heads=[(0, 0)], qblocks=qb)
+    unq = O.forward(prep, vf, sel, heads=[(0, 0)], qblocks=qb, quant=False)
+    assert_output_close(o[:, :1], ref, unq)
