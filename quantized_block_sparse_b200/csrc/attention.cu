@@ -82,10 +82,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 // then <= 2^24, the row sum l <= 2^41 and O stays far from fp32 overflow; the exact tile
 // max is computed only on that rare path (and on a row's first tile, where m = -inf).
 constexpr float kPsumLimit = 16777216.0f;
-// Of every 64-key tile a softmax thread holds 2 rows x 16 keys, in 8 groups ("reps") of
-// 2 keys per row; the first kPolyReps groups take exp2 on the FMA pipe (exp2_poly2), the rest
-// on the SFU (ex2.approx). Raising it moves exponentials off the SFU when that is the limit.
-constexpr int kPolyReps = 0;
 
 // Written by the TMA producer for every union step next to its K tile, read by the MMA
 // issuer and the softmax warps after they observe the slot's k_full phase (mbarrier
@@ -164,29 +160,6 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
 constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
 constexpr int kMagicBits = 0x4B400000;
 
-// 2^x on the FMA pipe for two values, x <= ~9 (scores minus the running max, log2 units).
-// Cody-Waite style range reduction x = n + f, n = rint(x), f in [-1/2, 1/2], then a
-// degree-3 polynomial for 2^f fitted for minimum relative error on [-1/2, 1/2] (max
-// relative error 7.5e-5, far below the bf16 rounding P receives), and n added to the
-// exponent field. x is clamped at -125 so the exponent stays normal; 2^-125 is negligible
-// next to a row sum >= 1.
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
-  const uint64_t x = f2pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-  const uint64_t t = add2(x, f2pack(kMagic, kMagic));      // 1.5*2^23 + rint(x)
-  const uint64_t n = add2(t, f2pack(-kMagic, -kMagic));    // rint(x), exact
-  const uint64_t f = fma2(n, f2pack(-1.f, -1.f), x);       // x - rint(x), exact
-  uint64_t p = fma2(f2pack(0.0551716648042202f, 0.0551716648042202f), f,
-                    f2pack(0.2426111400127411f, 0.2426111400127411f));
-  p = fma2(p, f, f2pack(0.6932609677314758f, 0.6932609677314758f));
-  p = fma2(p, f, f2pack(0.9999280571937561f, 0.9999280571937561f));
-  float p0, p1, t0, t1;
-  f2unpack(p, p0, p1);
-  f2unpack(t, t0, t1);
-  // (bits(t) << 23) == rint(x) << 23 (mod 2^32): the constant's low 9 bits are zero.
-  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
 // ---- TMEM access in the 16-lane shapes. For a 16-lane group starting at TMEM lane LB,
 // thread t of the warp holds rows LB + t/4 and LB + t/4 + 8:
 //   16x256b (8 columns per repetition k): regs 4k..4k+3 = (row0, 8k+2q), (row0, 8k+2q+1),
@@ -255,15 +228,10 @@ __device__ __forceinline__ void softmax_tile(const float (&A)[32], float sc, flo
     float a0, a1, b0, b1, pa0, pa1, pb0, pb1;
     f2unpack(x0, a0, a1);
     f2unpack(x1, b0, b1);
-    if (k < kPolyReps) {
-      exp2_poly2(a0, a1, pa0, pa1);
-      exp2_poly2(b0, b1, pb0, pb1);
-    } else {
-      pa0 = ex2_approx(a0);
-      pa1 = ex2_approx(a1);
-      pb0 = ex2_approx(b0);
-      pb1 = ex2_approx(b1);
-    }
+    pa0 = ex2_approx(a0);
+    pa1 = ex2_approx(a1);
+    pb0 = ex2_approx(b0);
+    pb1 = ex2_approx(b1);
     if (RAGGED) {
       const int c = 8 * k + 2 * q;
       if (c >= nvalid) pa0 = pb0 = 0.f;
