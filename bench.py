@@ -85,6 +85,27 @@ def profiled_traffic(workload: str):
     return int(fields["dram_bytes_per_launch"])
 
 
+def probe_ex2_rates(dev, iters=2048):
+    """The SFU exponential rate of this GPU, measured by the library's probe kernel (one CTA
+    per SM, 8 independent chains of dependent exponentials per thread, SM cycles read on the
+    device): per form, the median over the CTAs of exponentials per SM clock, and the number
+    of distinct SMs the CTAs ran on. Form 0 is ex2.approx.ftz.f32 (the kernels' form), forms 1
+    and 2 ex2.approx.f16x2 and ex2.approx.ftz.bf16x2 (two exponentials per instruction)."""
+    import torch
+
+    from quantized_block_sparse_b200 import sagesla as S
+    n = torch.cuda.get_device_properties(dev).multi_processor_count
+    out = torch.zeros(3 * n, dtype=torch.int64, device=dev)
+    res = {}
+    for form in (0, 1, 2):
+        S.sagesla_probe_ex2(form, 64, out)  # warm-up (module load, clocks)
+        S.sagesla_probe_ex2(form, iters, out)
+        torch.cuda.synchronize(dev)
+        a = out.view(n, 3).cpu().numpy()
+        res[form] = (float(np.median(a[:, 0] / a[:, 1])), int(len(set(a[:, 2].tolist()))))
+    return res
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -453,6 +474,13 @@ def run_ours(args, wl):
     # second denominator: the tcgen05 probe rate at the SM clock sampled during the run
     sm_mhz = clk.get("sm_mhz") or 1965.0
     peak_probe = PROBE_BF16_MAC_PER_CLK_SM * 2 * N_SM * sm_mhz * 1e6 / 1e12
+    # SFU floor of the attention kernel: one exponential per (query row, key) of every
+    # executed critical pair, plus phi(Q~) of the linear term (one per element of Q, an upper
+    # bound: phi takes the exponential only for x <= 0), over the probed ex2 rate
+    rates = probe_ex2_rates(dev)
+    exps = pairs * 64.0 * 64.0 + (wl.B * wl.H * float(wl.N) * wl.d if m > 0 else 0.0)
+    sfu_peak = rates[0][0] * N_SM * sm_mhz * 1e6 / 1e9  # Gexp/s
+    sfu_achieved = exps / (att_ms * 1e-3) / 1e9
     # forward-level roofline: every executed block of sagesla_forward on the tensor pipe
     fwd = forward_work(wl, nB, k_c, m)
     t_roof_s = fwd["int8_ops"] / (INT8_TO_BF16_RATE * peak * 1e12) + fwd["bf16_flops"] / (peak * 1e12)
@@ -481,6 +509,16 @@ def run_ours(args, wl):
                               f"MAC/clk/SM x 2 x {N_SM} SMs x the sampled SM clock; traffic = DRAM bytes "
                               f"per launch from the committed ncu summary (null once the kernel source "
                               f"differs from the profiled one)")},
+        "roofline_sfu": {"kernel": "attn_kernel", "bound": "sfu", "exps": exps,
+                         "achieved": sfu_achieved, "peak": sfu_peak, "unit": "Gexp/s",
+                         "frac": sfu_achieved / sfu_peak, "t_sfu_ms": exps / (sfu_peak * 1e9) * 1e3,
+                         "ex2_f32_per_clk_sm": rates[0][0], "ex2_f16x2_per_clk_sm": rates[1][0],
+                         "ex2_bf16x2_per_clk_sm": rates[2][0],
+                         "probe_sms": rates[0][1],
+                         "note": (f"exponentials: 4096 per executed 64x64 critical pair ({pairs}) + one "
+                                  f"per element of Q for phi(Q~) when m > 0 (upper bound); peak = the "
+                                  f"probed ex2.approx.ftz.f32 rate per SM clock (median over one CTA "
+                                  f"per SM) x {N_SM} SMs x the sampled SM clock")},
         "roofline_forward": {"bound": "tensor", "int8_ops": fwd["int8_ops"],
                              "bf16_flops": fwd["bf16_flops"], "t_roof_ms": t_roof_s * 1e3,
                              "fwd_ms": fwd_ms, "frac": t_roof_s * 1e3 / fwd_ms if fwd_ms else None,

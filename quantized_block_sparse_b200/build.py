@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsagesla.so")
 SOURCES = ["api.cu", "prepare.cu", "prepare_static.cu", "select.cu", "linear.cu", "attention.cu",
-           "selftest.cu", "w8a8.cu", "backward.cu"]
+           "selftest.cu", "probe.cu", "w8a8.cu", "backward.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",

@@ -60,6 +60,8 @@ def lib():
     L.sagesla_static_scratch_status.restype = ctypes.c_int
     L.sagesla_selftest_wait_timeout.argtypes = [_vp, ctypes.c_size_t, ctypes.c_uint, _vp]
     L.sagesla_selftest_wait_timeout.restype = ctypes.c_int
+    L.sagesla_probe_ex2.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+    L.sagesla_probe_ex2.restype = ctypes.c_int
     L.sagesla_backward_workspace_bytes.argtypes = [sp]
     L.sagesla_backward_workspace_bytes.restype = ctypes.c_size_t
     L.sagesla_backward.argtypes = ([sp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp,
@@ -272,6 +274,16 @@ def sagesla_selftest_wait_timeout(workspace, limit_us: int, stream=None):
     failure path of every kernel); sagesla_check_status then reports the timeout."""
     _check(lib().sagesla_selftest_wait_timeout(_ptr(workspace), workspace.numel(), int(limit_us),
                                                 _stream(stream)), "sagesla_selftest_wait_timeout")
+
+
+def sagesla_probe_ex2(form: int, iters: int, out, stream=None):
+    """Diagnostics: the SFU exponential-rate probe (form 0: ex2.approx.ftz.f32, 1: f16x2, 2: bf16x2)
+    on out.numel() // 3 CTAs; out is an int64 CUDA tensor that receives, per CTA, the
+    exponentials evaluated, the SM cycles taken and the SM id."""
+    assert out.dtype == torch.int64 and out.is_cuda and out.is_contiguous()
+    n = out.numel() // 3
+    _check(lib().sagesla_probe_ex2(int(form), int(iters), n, _ptr(out), out.numel(), _stream(stream)),
+           "sagesla_probe_ex2")
 
 
 class SageSLA:

@@ -133,6 +133,16 @@ def test_more_validation_paths(L):
     assert L.sagesla_selftest_wait_timeout(p, 128, 1000, None) == 1
     assert L.sagesla_selftest_wait_timeout(p, 1 << 20, 0, None) == 1
     assert L.sagesla_selftest_wait_timeout(p, 1 << 20, 1000001, None) == 1
+    # the SFU rate probe: form 0/1/2, iters in 1..2^20, 1..1024 CTAs, an aligned out of 3 per CTA
+    assert L.sagesla_probe_ex2(3, 64, 4, p, 12, None) == 1
+    assert L.sagesla_probe_ex2(-1, 64, 4, p, 12, None) == 1
+    assert L.sagesla_probe_ex2(0, 0, 4, p, 12, None) == 1
+    assert L.sagesla_probe_ex2(0, (1 << 20) + 1, 4, p, 12, None) == 1
+    assert L.sagesla_probe_ex2(1, 64, 0, p, 12, None) == 1
+    assert L.sagesla_probe_ex2(1, 64, 1025, p, 3 * 1025, None) == 1
+    assert L.sagesla_probe_ex2(0, 64, 4, None, 12, None) == 1
+    assert L.sagesla_probe_ex2(0, 64, 4, ctypes.c_void_p(0x1004), 12, None) == 1
+    assert L.sagesla_probe_ex2(0, 64, 4, p, 11, None) == 1
     # the marginal sums on their own: m in 0..nB-1, aligned pointers, a large enough workspace
     # (shape N = 1024: nB = 16)
     assert L.sagesla_marginal_sums(ctypes.byref(sh), p, -1, p, p, p, p, p, big, None) == 1
