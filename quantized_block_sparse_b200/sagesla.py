@@ -98,6 +98,12 @@ def _shape(B, H, N, d=HEAD_DIM):
     return _Shape(int(B), int(H), int(N), int(d))
 
 
+def _require(ok: bool, what: str):
+    """Argument check of the binding (kept under python -O)."""
+    if not ok:
+        raise SageSLAError(f"invalid argument: {what}")
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -177,7 +183,8 @@ def sagesla_prepare(q, k, v, workspace, sm_scale=None, out: Prepared | None = No
     """Steps 1-3 (+ block means and linear states). q, k, v: bf16 [B,H,N,128] on the GPU."""
     B, H, N, d, nB = _dims(q)
     for t in (q, k, v):
-        assert t.dtype == torch.bfloat16 and t.is_cuda and t.is_contiguous() and t.shape == q.shape
+        _require(t.dtype == torch.bfloat16 and t.is_cuda and t.is_contiguous() and t.shape == q.shape,
+                 "inputs must be contiguous bf16 CUDA tensors of one shape")
     if out is None:
         out = alloc_prepared(B, H, N, q.device)
     c_s = softmax_scale(d) if sm_scale is None else float(sm_scale)
@@ -195,7 +202,8 @@ def sagesla_prepare_static_scratch(q, k, v, sm_scale=None, out: Prepared | None 
     Calls share that array, so order them on one stream."""
     B, H, N, d, nB = _dims(q)
     for t in (q, k, v):
-        assert t.dtype == torch.bfloat16 and t.is_cuda and t.is_contiguous() and t.shape == q.shape
+        _require(t.dtype == torch.bfloat16 and t.is_cuda and t.is_contiguous() and t.shape == q.shape,
+                 "inputs must be contiguous bf16 CUDA tensors of one shape")
     if out is None:
         out = alloc_prepared(B, H, N, q.device)
     c_s = softmax_scale(d) if sm_scale is None else float(sm_scale)
@@ -256,7 +264,8 @@ def sagesla_marginal_sums(mask, m, h, z, workspace, N=None, stream=None):
     z fp32 [B,H,nB,128], N the token count (default 64 nB) -> (H bf16 like h, Z fp32 like z)."""
     B, H, nB = h.shape[:3]
     N = 64 * nB if N is None else int(N)
-    assert h.dtype == torch.bfloat16 and z.dtype == torch.float32 and mask.dtype == torch.bfloat16
+    _require(h.dtype == torch.bfloat16 and z.dtype == torch.float32 and mask.dtype == torch.bfloat16,
+             "h bf16, z fp32 and mask bf16")
     Hout = torch.empty_like(h)
     Zout = torch.empty_like(z)
     _check(lib().sagesla_marginal_sums(ctypes.byref(_shape(B, H, N, HEAD_DIM)), _ptr(mask), int(m), _ptr(h),
@@ -280,7 +289,8 @@ def sagesla_probe_ex2(form: int, iters: int, out, stream=None):
     """Diagnostics: the SFU exponential-rate probe (form 0: ex2.approx.ftz.f32, 1: f16x2, 2: bf16x2)
     on out.numel() // 3 CTAs; out is an int64 CUDA tensor that receives, per CTA, the
     exponentials evaluated, the SM cycles taken and the SM id."""
-    assert out.dtype == torch.int64 and out.is_cuda and out.is_contiguous()
+    _require(out.dtype == torch.int64 and out.is_cuda and out.is_contiguous(),
+             "out: contiguous int64 CUDA tensor")
     n = out.numel() // 3
     _check(lib().sagesla_probe_ex2(int(form), int(iters), n, _ptr(out), out.numel(), _stream(stream)),
            "sagesla_probe_ex2")
@@ -312,7 +322,8 @@ class SageSLA:
 # ---------------------------------------------------------------- W8A8 linear layer
 def sagesla_w8a8_quantize(x, stream=None):
     """bf16 [rows, K] -> (int8 codes [rows, K], fp32 scales [ceil(rows/128), ceil(K/128)])."""
-    assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and x.dim() == 2
+    _require(x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and x.dim() == 2,
+             "x: contiguous 2-D bf16 CUDA tensor")
     R, K = x.shape
     x8 = torch.empty(R, K, dtype=torch.int8, device=x.device)
     s = torch.empty(-(-R // 128), -(-K // 128), dtype=torch.float32, device=x.device)
@@ -341,7 +352,8 @@ def sagesla_backward(q, k, v, dout, prep: Prepared, sel: Selection, sm_scale=Non
     with the block lists of `sel` held fixed and the quantization read straight through."""
     B, H, N, d, nB = _dims(q)
     for t in (q, k, v, dout):
-        assert t.dtype == torch.bfloat16 and t.is_cuda and t.is_contiguous() and t.shape == q.shape
+        _require(t.dtype == torch.bfloat16 and t.is_cuda and t.is_contiguous() and t.shape == q.shape,
+                 "inputs must be contiguous bf16 CUDA tensors of one shape")
     sh = _shape(B, H, N, d)
     if workspace is None:
         n = lib().sagesla_backward_workspace_bytes(ctypes.byref(sh))

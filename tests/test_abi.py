@@ -163,3 +163,14 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(S, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(S.SageSLAError):
         S.lib()
+
+
+def test_binding_rejects_host_tensors_before_any_call():
+    import torch
+    q = torch.zeros(1, 1, 64, 128, dtype=torch.bfloat16)  # host memory: not a CUDA tensor
+    with pytest.raises(S.SageSLAError, match="invalid argument"):
+        S.sagesla_prepare(q, q, q, workspace=None)
+    with pytest.raises(S.SageSLAError, match="invalid argument"):
+        S.sagesla_w8a8_quantize(q[0, 0])
+    with pytest.raises(S.SageSLAError, match="invalid argument"):
+        S.sagesla_probe_ex2(0, 64, torch.zeros(3, dtype=torch.int64))
