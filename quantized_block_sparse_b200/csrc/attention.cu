@@ -318,12 +318,44 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   const int pr = blockIdx.x, bh = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nB = p.nB;
-  int tile = pr, seg = 0;  // tile pr of the head: entry tile of segment seg
+  // Tile pr of the head is entry `tile` of segment `seg`. Every warp finds it at once, with
+  // one round of loads instead of a chain of dependent ones: lane l holds the tile counts of
+  // segments 4l..4l+3 (n_seg <= 128), an inclusive warp scan of their sums gives each lane
+  // its range of tiles, and the lane whose range holds pr walks its four segments.
+  int tile = pr, seg = 0;
   {
     const int* cnt = p.pair_counts + static_cast<size_t>(bh) * p.n_seg;
-    while (seg < p.n_seg && tile >= __ldg(cnt + seg)) tile -= __ldg(cnt + seg++);
+    int c[4], own = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      c[u] = 4 * lane + u < p.n_seg ? __ldg(cnt + 4 * lane + u) : 0;
+      own += c[u];
+    }
+    int incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, pr >= incl - own && pr < incl);
+    if (hit == 0u) return;  // past the head's last tile (whole CTA, before any barrier)
+    const int src = __ffs(hit) - 1;
+    tile = pr - __shfl_sync(0xffffffffu, incl - own, src);
+    seg = 4 * src;
+    bool found = false;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int cu = __shfl_sync(0xffffffffu, c[u], src);
+      if (!found) {
+        if (tile < cu) {
+          seg = 4 * src + u;
+          found = true;
+        } else {
+          tile -= cu;
+        }
+      }
+    }
   }
-  if (seg >= p.n_seg) return;  // past the head's last tile (whole CTA, before any barrier)
   const int2 pq = p.pairs[static_cast<size_t>(bh) * nB + seg * kPairSegment + tile];
   const int i0 = pq.x, i1 = pq.y;  // the pair (i1 = -1: block i0 alone)
   // Linear branch: H_i0 (and H_i1) enter the V ring after the last V tile as 16 KB chunks
@@ -989,6 +1021,7 @@ cudaError_t launch_attention(const Dims& g, const void* q, float sm_scale, const
   int2* pairs = reinterpret_cast<int2*>(ws + L.pairs);
   int* pair_counts = reinterpret_cast<int*>(ws + L.pair_counts);
   int n_seg = (g.nB + kPairSegment - 1) / kPairSegment;
+  if (n_seg > 128) return cudaErrorInvalidValue;  // attn_kernel's tile lookup: 4 segments per lane
   if (whole_head_pairing(g)) {  // pairs over the whole head, one segment
     n_seg = 1;
     uint8_t* win = reinterpret_cast<uint8_t*>(ws + L.pair_window);
