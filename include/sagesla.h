@@ -240,10 +240,10 @@ int sagesla_selftest_wait_timeout(void* workspace, size_t workspace_bytes,
  * for more than half of an SM's shared memory so that no two share an SM; every thread runs
  * 8 independent chains of `iters` dependent exponentials (x <- 2^-x) in the form `form`:
  * 0 = ex2.approx.ftz.f32 (the form the kernels use), 1 = ex2.approx.f16x2, 2 =
- * ex2.approx.ftz.bf16x2 (forms 1 and 2: two 16-bit exponentials per instruction). CTA b writes three values to out (device memory, caller-
- * owned, out_len >= 3 * n_ctas): out[3b] = exponentials it evaluated, out[3b+1] = SM clock
- * cycles (clock64) around its loop, out[3b+2] = the SM it ran on. exponentials / cycles is
- * the rate per clock of one SM. Asynchronous on `stream`. Returns SAGESLA_ERR_INVALID_ARG
+ * ex2.approx.ftz.bf16x2 (forms 1 and 2: two 16-bit exponentials per instruction). CTA b
+ * writes three values to out (device memory, caller-owned, out_len >= 3 * n_ctas):
+ * out[3b] = exponentials it evaluated, out[3b+1] = SM clock cycles (clock64) around its
+ * loop, out[3b+2] = the SM it ran on. exponentials / cycles is the rate per clock of one SM. Asynchronous on `stream`. Returns SAGESLA_ERR_INVALID_ARG
  * for form not 0/1/2, iters outside [1, 2^20], n_ctas outside [1, 1024], a NULL or
  * misaligned out or a short out_len, SAGESLA_ERR_CUDA if the launch failed. */
 int sagesla_probe_ex2(int form, int iters, int n_ctas, unsigned long long* out, size_t out_len,
